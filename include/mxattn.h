@@ -1,0 +1,209 @@
+/*
+ * mxattn.h -- C ABI of libmxattn.so: MXAttention's MXFP4 forward attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+ * Quantization for MXFP4 Attention", as described on its Pith review page and
+ * in the 10100.com article) computes, per attention head:
+ *   1. a fixed orthonormal Hadamard rotation of every Q and K row (Fig. 1;
+ *      axioms ledger, Sec. 4.3);
+ *   2. MXFP4 quantization of Q, K and V: groups of 32 values share one E8M0
+ *      power-of-two scale, each value becomes an E2M1 code (grid 0, +-0.5,
+ *      +-1, +-1.5, +-2, +-3, +-4, +-6; round to nearest, ties to even,
+ *      saturating at 6).  The scale exponent is the Universal Optimal
+ *      Scaling ceiling rule with boundary Qmax = 7.25 (Fig. 3: the block
+ *      maximum maps to (3.625, 7.25]); Qmax = 6 and the OCP floor rule are
+ *      ablation options.  Q/K groups run along the head dimension, V groups
+ *      along the key axis;
+ *   3. a FlashAttention-2 style online softmax with Pre-Normalization
+ *      Quantization (Fig. 4): every unnormalized exponential tile
+ *      P~ = exp(S - m_running) is quantized to MXFP4 once and that same
+ *      quantized tile feeds both the row sum l and the P~ V update.
+ *
+ * Conventions
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library allocates no memory, never synchronizes (except
+ *    mxattn_get_device_error), and enqueues all work on `stream`, a
+ *    cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Arguments are validated before anything is enqueued; an invalid call
+ *    returns an error status and enqueues nothing.
+ *  - q, k, v, out are contiguous [B, H, N, d] ("BHND") in opts->dtype; out
+ *    has the input dtype.  Self-attention without masking, N_q = N_k = N.
+ *  - Codes are packed two per byte, element 2i in the LOW nibble, element
+ *    2i+1 in the high nibble; bit 3 of a code is the sign (a negative value
+ *    that rounds to zero keeps its sign: code 0x8).  Scales are E8M0 bytes
+ *    (2^(byte-127)); the byte 0xFF is never written; an all-zero group gets
+ *    byte 0x00 and zero codes.
+ *
+ * Packed attention-operand layouts (what mxattn_hadamard_quant_qk and
+ * mxattn_quant_v write, what mxattn_attention_mxfp4 reads).  They are the
+ * shared-memory images the tcgen05 block-scaled MMA consumes, so each tile is
+ * moved with one bulk copy:
+ *
+ *  QK codes   [B*H][T128][128][d/2] bytes, T128 = ceil(N/128).  Tile t holds
+ *             tokens 128t .. 128t+127 (rows past N are zero).  Row r of a
+ *             tile is stored at byte r*(d/2); its 16-byte chunk c (= MX group
+ *             c, elements 32c..32c+31) is stored at chunk position c ^ s(r):
+ *               d = 128:  s(r) = (r >> 1) & 3     (64-byte swizzle)
+ *               d =  64:  s(r) = (r >> 2) & 1     (32-byte swizzle)
+ *  QK scales  [B*H][T128][512] bytes, one 512-byte scale atom per 128-row
+ *             tile: the scale of token r (0..127 within the tile), group g
+ *             (0..3) sits at byte (r % 32)*16 + (r / 32)*4 + g.  Groups
+ *             g >= d/32 are zero.
+ *  V codes    [B*H][T64][d][32] bytes, T64 = ceil(N/64): V is transposed so
+ *             that each channel is a row of 64 keys (32 bytes).  Row c of
+ *             tile j holds keys 64j .. 64j+63 of channel c; its 16-byte chunk
+ *             h (keys 64j+32h .. +31, one MX group) sits at chunk position
+ *             h ^ ((c >> 2) & 1).  Keys past N are zero.
+ *  V scales   [B*H][T128][512] bytes: the atom of keys 128t .. 128t+127 holds
+ *             the scale of channel c, key group g (0..3) at byte
+ *             (c % 32)*16 + (c / 32)*4 + g.  Channels >= d are zero.
+ *
+ * Workspace (mxattn_forward, mxattn_attention_mxfp4): opts->workspace is a
+ * device buffer of at least mxattn_workspace_bytes() bytes, 256-byte aligned.
+ * Its first 256 bytes are a status block that the kernels set when a bounded
+ * device-side wait expires; zero it once with mxattn_workspace_init before
+ * first use.  mxattn_forward keeps the packed Q/K/V operands after it.
+ */
+#ifndef MXATTN_H_
+#define MXATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MXATTN_ABI_VERSION 1
+
+typedef enum mxattn_status {
+  MXATTN_OK = 0,
+  MXATTN_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad option value        */
+  MXATTN_ERR_UNSUPPORTED = 2, /* valid but not implemented (d, key_tile, dtype)   */
+  MXATTN_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned       */
+  MXATTN_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed              */
+  MXATTN_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (see below)   */
+} mxattn_status;
+
+typedef enum mxattn_scale_rule {
+  MXATTN_SCALE_UOS = 0,        /* ceiling rule, boundary 29/4: max -> (3.625, 7.25] */
+  MXATTN_SCALE_QMAX6 = 1,      /* ceiling rule, boundary 6:    max -> (3, 6]        */
+  MXATTN_SCALE_OCP = 2,        /* OCP floor rule e = floor(log2 amax) - 2: [4, 8)  */
+  MXATTN_SCALE_CEIL_CUSTOM = 3 /* ceiling rule, boundary opts.qmax (> 0, finite)   */
+} mxattn_scale_rule;
+
+typedef enum mxattn_dtype { MXATTN_BF16 = 0, MXATTN_FP32 = 1 } mxattn_dtype;
+
+typedef struct mxattn_opts {
+  int scale_rule;          /* mxattn_scale_rule, used for Q, K, V and the P~ tiles      */
+  float qmax;              /* boundary for MXATTN_SCALE_CEIL_CUSTOM                      */
+  int pnq;                 /* 1: l from the quantized tile (PNQ); 0: direct placement   */
+  int rotate;              /* 1: Hadamard-rotate Q and K before quantizing               */
+  int dtype;               /* mxattn_dtype of q, k, v, out                               */
+  int key_tile;            /* keys per online-softmax step; 64 is supported             */
+  float rescale_tau;       /* the running max moves only when it grows by more than    */
+                           /* tau (log2 units); 0 = eager FlashAttention-2 update       */
+  void* workspace;         /* device buffer, see mxattn_workspace_bytes                  */
+  size_t workspace_bytes;  /* its size in bytes                                          */
+} mxattn_opts;
+
+/* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
+ * key_tile 64, rescale_tau 8, no workspace. */
+void mxattn_opts_default(mxattn_opts* opts);
+
+/* Bytes of workspace mxattn_forward needs for this problem (status block plus
+ * packed Q, K, V operands); 0 for invalid sizes. */
+size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts);
+
+/* Sizes of the packed attention operands described above (0 for invalid sizes). */
+size_t mxattn_qk_codes_bytes(int B, int H, int N, int d);
+size_t mxattn_qk_scales_bytes(int B, int H, int N, int d);
+size_t mxattn_v_codes_bytes(int B, int H, int N, int d);
+size_t mxattn_v_scales_bytes(int B, int H, int N, int d);
+
+/* Zero the workspace status block (enqueued on stream). */
+mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* stream);
+
+/*
+ * Generic MXFP4 quantization of a row-major [rows][cols] matrix x
+ * (opts->dtype), with the scale rule of opts (10100.com article: 32-element
+ * groups sharing one E8M0 scale; Fig. 3 of the paper for the rules).
+ *  group_axis 0: groups of 32 consecutive columns of each row;
+ *                codes [rows][ceil(cols/32)*16], scales [rows][ceil(cols/32)].
+ *  group_axis 1: groups of 32 consecutive rows of each column, written
+ *                transposed: codes [cols][ceil(rows/32)*16],
+ *                scales [cols][ceil(rows/32)].
+ * Partial tail groups are zero-padded.  No rotation is applied.
+ */
+mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, int group_axis,
+                                    const mxattn_opts* opts, uint8_t* codes, uint8_t* scales,
+                                    void* stream);
+
+/*
+ * Step 1+2 for Q and K: Hadamard rotation (if opts->rotate) and MXFP4
+ * quantization along d, written in the packed QK operand layout.
+ * The rotation is y = x H_d / sqrt(d) for the natural-order Sylvester
+ * Hadamard matrix, computed in fp32 as log2(d) butterfly stages
+ * h = 1, 2, ..., d/2 ((a, b) -> (a + b, a - b)) followed by one multiply by
+ * fl32(1/sqrt(d)); the scale rule reads these fp32 values.
+ * d in {64, 128}.  Buffers: mxattn_qk_codes_bytes / mxattn_qk_scales_bytes.
+ */
+mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
+                                       const mxattn_opts* opts, uint8_t* q_codes,
+                                       uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales,
+                                       void* stream);
+
+/*
+ * Step 2 for V: MXFP4 quantization in groups of 32 consecutive keys per
+ * channel (no rotation), written in the packed V operand layout.
+ */
+mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mxattn_opts* opts,
+                             uint8_t* v_codes, uint8_t* v_scales, void* stream);
+
+/*
+ * Step 3 alone on packed operands: S = Q^ K^T (block-scaled FP4 tensor-core
+ * MMA, fp32 accumulation) times softmax_scale, online softmax over key tiles
+ * of opts->key_tile keys, each exponential tile quantized to MXFP4 in groups
+ * of 32 keys with the scale rule of opts, l updated from the quantized tile
+ * (PNQ) or from the unquantized one (pnq = 0), O~ += P^ V^, O = O~ / l in
+ * opts->dtype.  Requires opts->workspace (status block, >= 256 bytes).
+ */
+mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+                                     const uint8_t* k_codes, const uint8_t* k_scales,
+                                     const uint8_t* v_codes, const uint8_t* v_scales, int B, int H,
+                                     int N, int d, float softmax_scale, const mxattn_opts* opts,
+                                     void* out, void* stream);
+
+/*
+ * The whole forward pass: mxattn_hadamard_quant_qk + mxattn_quant_v into
+ * the workspace, then mxattn_attention_mxfp4.  d in {64, 128}, N >= 1.
+ */
+mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B, int H, int N,
+                             int d, float softmax_scale, const mxattn_opts* opts, void* out,
+                             void* stream);
+
+/*
+ * Synchronize `stream`, read the workspace status block and clear it.
+ * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
+ * last call (its output is then undefined), MXATTN_OK otherwise.
+ */
+mxattn_status mxattn_get_device_error(const mxattn_opts* opts, void* stream);
+
+/* Static string naming a status code. */
+const char* mxattn_status_string(mxattn_status status);
+
+/*
+ * Dense FP4 tensor-core throughput probe (not part of the method): `ctas`
+ * CTAs each issue `iters` back-to-back tcgen05 kind::mxf4 block-scaled MMAs
+ * of shape M=128 x n x K=64 from shared memory into tensor memory.
+ * n in {64, 128, 256}.  The caller times the launch; flops = ctas * iters *
+ * 2 * 128 * n * 64.
+ */
+mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXATTN_H_ */

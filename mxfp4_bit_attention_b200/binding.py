@@ -1,0 +1,227 @@
+"""ctypes binding of libmxattn.so (declared in include/mxattn.h).
+
+Argument marshalling only: torch tensors become device pointers and sizes,
+the stream is torch's current CUDA stream, and every step of the method runs
+in the library's kernels.  There is no fallback: if the library cannot be
+loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+SCALE_UOS, SCALE_QMAX6, SCALE_OCP, SCALE_CEIL_CUSTOM = 0, 1, 2, 3
+BF16, FP32 = 0, 1
+
+STATUS = {0: "MXATTN_OK", 1: "MXATTN_ERR_INVALID_ARG", 2: "MXATTN_ERR_UNSUPPORTED",
+          3: "MXATTN_ERR_WORKSPACE", 4: "MXATTN_ERR_CUDA", 5: "MXATTN_ERR_TIMEOUT"}
+
+EXPORTS = (
+    "mxattn_opts_default", "mxattn_workspace_bytes", "mxattn_qk_codes_bytes",
+    "mxattn_qk_scales_bytes", "mxattn_v_codes_bytes", "mxattn_v_scales_bytes",
+    "mxattn_workspace_init", "mxattn_quantize_mxfp4", "mxattn_hadamard_quant_qk",
+    "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
+    "mxattn_status_string", "mxattn_fp4_mma_probe",
+)
+
+
+class MXAttnError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class COpts(ctypes.Structure):
+    _fields_ = [("scale_rule", ctypes.c_int), ("qmax", ctypes.c_float), ("pnq", ctypes.c_int),
+                ("rotate", ctypes.c_int), ("dtype", ctypes.c_int), ("key_tile", ctypes.c_int),
+                ("rescale_tau", ctypes.c_float), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+@dataclass
+class Opts:
+    scale_rule: int = SCALE_UOS
+    qmax: float = 7.25
+    pnq: bool = True
+    rotate: bool = True
+    key_tile: int = 64
+    rescale_tau: float = 8.0
+
+
+def lib_path() -> str:
+    return os.path.join(HERE, "libmxattn.so")
+
+
+_lib = None
+
+
+def load():
+    """Load libmxattn.so once; raise if it is missing or lacks a symbol."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m mxfp4_bit_attention_b200.build`")
+    L = ctypes.CDLL(path)
+    P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    PO = ctypes.POINTER(COpts)
+    sig = {
+        "mxattn_opts_default": ([PO], None),
+        "mxattn_workspace_bytes": ([i32, i32, i32, i32, PO], sz),
+        "mxattn_qk_codes_bytes": ([i32, i32, i32, i32], sz),
+        "mxattn_qk_scales_bytes": ([i32, i32, i32, i32], sz),
+        "mxattn_v_codes_bytes": ([i32, i32, i32, i32], sz),
+        "mxattn_v_scales_bytes": ([i32, i32, i32, i32], sz),
+        "mxattn_workspace_init": ([PO, P], i32),
+        "mxattn_quantize_mxfp4": ([P, i64, i64, i32, PO, P, P, P], i32),
+        "mxattn_hadamard_quant_qk": ([P, P, i32, i32, i32, i32, PO, P, P, P, P, P], i32),
+        "mxattn_quant_v": ([P, i32, i32, i32, i32, PO, P, P, P], i32),
+        "mxattn_attention_mxfp4": ([P, P, P, P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_forward": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_get_device_error": ([PO, P], i32),
+        "mxattn_status_string": ([i32], ctypes.c_char_p),
+        "mxattn_fp4_mma_probe": ([i32, i32, i32, P], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def _check(call, status):
+    if status != 0:
+        raise MXAttnError(call, status)
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _copts(o: Opts | None, dtype: int, workspace=None) -> COpts:
+    o = o or Opts()
+    c = COpts()
+    load().mxattn_opts_default(ctypes.byref(c))
+    c.scale_rule, c.qmax, c.pnq, c.rotate = int(o.scale_rule), float(o.qmax), int(bool(o.pnq)), int(bool(o.rotate))
+    c.dtype, c.key_tile, c.rescale_tau = dtype, int(o.key_tile), float(o.rescale_tau)
+    if workspace is not None:
+        c.workspace = ctypes.c_void_p(workspace.data_ptr())
+        c.workspace_bytes = workspace.numel() * workspace.element_size()
+    return c
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def operand_sizes(B: int, H: int, N: int, d: int) -> dict:
+    L = load()
+    return {"q_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "q_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
+            "k_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "k_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
+            "v_codes": L.mxattn_v_codes_bytes(B, H, N, d), "v_scales": L.mxattn_v_scales_bytes(B, H, N, d)}
+
+
+def mxattn_workspace_bytes(B: int, H: int, N: int, d: int, opts: Opts | None = None) -> int:
+    c = _copts(opts, BF16)
+    return int(load().mxattn_workspace_bytes(B, H, N, d, ctypes.byref(c)))
+
+
+def new_workspace(B, H, N, d, opts=None, device="cuda"):
+    """A zeroed workspace tensor (uint8) of the size mxattn_forward needs."""
+    import torch
+    return torch.zeros(mxattn_workspace_bytes(B, H, N, d, opts), dtype=torch.uint8, device=device)
+
+
+def mxattn_quantize_mxfp4(x, group_axis=0, opts: Opts | None = None, codes=None, scales=None, stream=None):
+    """Plain MXFP4 quantization of a 2-D bf16/fp32 tensor; returns (codes, scales) uint8."""
+    import torch
+    rows, cols = x.shape
+    outer, inner = (rows, cols) if group_axis == 0 else (cols, rows)
+    ng = (inner + 31) // 32
+    codes = codes if codes is not None else torch.empty((outer, ng * 16), dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else torch.empty((outer, ng), dtype=torch.uint8, device=x.device)
+    c = _copts(opts, _dtype_code(x))
+    _check("mxattn_quantize_mxfp4", load().mxattn_quantize_mxfp4(
+        _ptr(x), rows, cols, group_axis, ctypes.byref(c), _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def _alloc_operands(B, H, N, d, device):
+    import torch
+    s = operand_sizes(B, H, N, d)
+    return {k: torch.empty(v, dtype=torch.uint8, device=device) for k, v in s.items()}
+
+
+def mxattn_hadamard_quant_qk(q, k, opts: Opts | None = None, out=None, stream=None):
+    """Rotate + quantize Q and K ([B, H, N, d]) into the packed QK operand layout."""
+    B, H, N, d = q.shape
+    out = out or _alloc_operands(B, H, N, d, q.device)
+    c = _copts(opts, _dtype_code(q))
+    _check("mxattn_hadamard_quant_qk", load().mxattn_hadamard_quant_qk(
+        _ptr(q), _ptr(k), B, H, N, d, ctypes.byref(c), _ptr(out["q_codes"]), _ptr(out["q_scales"]),
+        _ptr(out["k_codes"]), _ptr(out["k_scales"]), _stream(stream)))
+    return out
+
+
+def mxattn_quant_v(v, opts: Opts | None = None, out=None, stream=None):
+    """Quantize V ([B, H, N, d]) along keys into the packed V operand layout."""
+    B, H, N, d = v.shape
+    out = out or _alloc_operands(B, H, N, d, v.device)
+    c = _copts(opts, _dtype_code(v))
+    _check("mxattn_quant_v", load().mxattn_quant_v(
+        _ptr(v), B, H, N, d, ctypes.byref(c), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _stream(stream)))
+    return out
+
+
+def mxattn_attention_mxfp4(ops, B, H, N, d, softmax_scale, out, opts: Opts | None = None, workspace=None,
+                           stream=None):
+    """Fused MXFP4 attention on packed operands (dict from the two quantizers)."""
+    import torch
+    ws = workspace if workspace is not None else torch.zeros(256, dtype=torch.uint8, device=out.device)
+    c = _copts(opts, _dtype_code(out), ws)
+    _check("mxattn_attention_mxfp4", load().mxattn_attention_mxfp4(
+        _ptr(ops["q_codes"]), _ptr(ops["q_scales"]), _ptr(ops["k_codes"]), _ptr(ops["k_scales"]),
+        _ptr(ops["v_codes"]), _ptr(ops["v_scales"]), B, H, N, d, float(softmax_scale), ctypes.byref(c),
+        _ptr(out), _stream(stream)))
+    return out
+
+
+def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None, stream=None):
+    """MXAttention forward: O = MXFP4-PNQ-attention(Q, K, V) for [B, H, N, d] tensors."""
+    import torch
+    B, H, N, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    out = out if out is not None else torch.empty_like(q)
+    ws = workspace if workspace is not None else new_workspace(B, H, N, d, opts, q.device)
+    c = _copts(opts, _dtype_code(q), ws)
+    _check("mxattn_forward", load().mxattn_forward(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def mxattn_get_device_error(workspace, stream=None) -> int:
+    """Synchronize, read and clear the workspace status block; returns the status code."""
+    c = _copts(None, BF16, workspace)
+    return int(load().mxattn_get_device_error(ctypes.byref(c), _stream(stream)))
+
+
+def mxattn_fp4_mma_probe(ctas: int, iters: int, n: int, stream=None):
+    _check("mxattn_fp4_mma_probe", load().mxattn_fp4_mma_probe(ctas, iters, n, _stream(stream)))

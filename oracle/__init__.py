@@ -1,0 +1,240 @@
+"""CPU oracle for MXAttention's MXFP4 forward attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never does, and this package imports nothing from it.
+
+``mxref.c`` holds the arithmetic (plain C, fp64 accumulation, fp32 where the
+method rounds to fp32); this module compiles it with gcc, loads it through
+ctypes and marshals numpy arrays.  ``uos_theory`` holds the data-free UOS
+objective, ``layout`` reads the CUDA library's packed operand layouts back into
+plain row-major arrays.
+
+Sources: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+Quantization for MXFP4 Attention" -- Pith review page (axioms ledger; Figs. 1,
+3, 4; Eq. (96)) and the 10100.com article (MXFP4 format, UOS, PNQ).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "mxref.c")
+LIB = os.path.join(HERE, "libmxref.so")
+
+RULE_UOS, RULE_QMAX6, RULE_OCP, RULE_CUSTOM = 0, 1, 2, 3
+RULES = {"uos": RULE_UOS, "qmax6": RULE_QMAX6, "ocp": RULE_OCP, "custom": RULE_CUSTOM}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile mxref.c into libmxref.so next to it (gcc, OpenMP, no FMA contraction)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        cmd = ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+               "-std=gnu11", "-o", LIB, SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return LIB
+
+
+class AttnCfg(ctypes.Structure):
+    _fields_ = [("key_tile", ctypes.c_int), ("pnq", ctypes.c_int), ("quant_p", ctypes.c_int),
+                ("rule", ctypes.c_int), ("qmax", ctypes.c_double), ("tau", ctypes.c_double)]
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(LIB)
+            P = ctypes.c_void_p
+            i64, i32, f64, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float
+            L.mxref_e2m1_decode.argtypes = [i32]
+            L.mxref_e2m1_decode.restype = f64
+            L.mxref_e2m1_encode.argtypes = [f64]
+            L.mxref_e2m1_encode.restype = i32
+            L.mxref_scale_exponent.argtypes = [f64, i32, f64]
+            L.mxref_scale_exponent.restype = i32
+            L.mxref_quantize.argtypes = [P, i64, i64, i32, i32, f64, P, P]
+            L.mxref_quantize.restype = None
+            L.mxref_fwht_row.argtypes = [P, i32]
+            L.mxref_fwht_row.restype = None
+            L.mxref_rotate_rows.argtypes = [P, i64, i32]
+            L.mxref_rotate_rows.restype = None
+            L.mxref_rotate_quantize_rows.argtypes = [P, i64, i32, i32, i32, f64, P, P]
+            L.mxref_rotate_quantize_rows.restype = None
+            L.mxref_dequantize.argtypes = [P, P, i64, P]
+            L.mxref_dequantize.restype = None
+            L.mxref_attention_rows.argtypes = [P, i64, P, P, i32, i32, f32, ctypes.POINTER(AttnCfg),
+                                               P, P, P, P, P]
+            L.mxref_attention_rows.restype = None
+            L.mxref_num_threads.argtypes = []
+            L.mxref_num_threads.restype = i32
+            _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def num_threads() -> int:
+    return int(lib().mxref_num_threads())
+
+
+# ----------------------------------------------------------------------------------------------
+# Element format and scale rule
+# ----------------------------------------------------------------------------------------------
+
+def e2m1_encode(v: float) -> int:
+    return int(lib().mxref_e2m1_encode(float(v)))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().mxref_e2m1_decode(int(code)))
+
+
+def scale_exponent(amax: float, rule: int = RULE_UOS, qmax: float = 7.25) -> int:
+    return int(lib().mxref_scale_exponent(float(amax), int(rule), float(qmax)))
+
+
+# ----------------------------------------------------------------------------------------------
+# Quantization
+# ----------------------------------------------------------------------------------------------
+
+def quantize(x: np.ndarray, axis: int = 0, rule: int = RULE_UOS, qmax: float = 7.25):
+    """MXFP4-quantize a 2-D fp32 matrix in groups of 32 along columns (axis 0)
+    or along rows (axis 1, output transposed).  Returns (codes, scales) with
+    codes unpacked, one 4-bit code per byte: [outer, ceil(inner/32)*32]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    outer, inner = (rows, cols) if axis == 0 else (cols, rows)
+    ng = (inner + 31) // 32
+    codes = np.zeros((outer, ng * 32), np.uint8)
+    scales = np.zeros((outer, ng), np.uint8)
+    lib().mxref_quantize(_ptr(x), rows, cols, axis, rule, qmax, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def rotate_rows(x: np.ndarray) -> np.ndarray:
+    """Hadamard-rotate each row (fp32, normalized by fl32(1/sqrt(d)))."""
+    y = np.array(x, dtype=np.float32, copy=True, order="C")
+    rows, d = y.reshape(-1, y.shape[-1]).shape
+    lib().mxref_rotate_rows(_ptr(y), rows, d)
+    return y
+
+
+def rotate_quantize_rows(x: np.ndarray, rotate: bool = True, rule: int = RULE_UOS, qmax: float = 7.25):
+    """Q/K operand: optional rotation then groups of 32 along d.
+    Returns unpacked codes [rows, d] and scales [rows, d/32]."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    d = x.shape[-1]
+    x2 = x.reshape(-1, d)
+    rows = x2.shape[0]
+    codes = np.zeros((rows, d), np.uint8)
+    scales = np.zeros((rows, d // 32), np.uint8)
+    lib().mxref_rotate_quantize_rows(_ptr(x2), rows, d, int(bool(rotate)), rule, qmax, _ptr(codes),
+                                     _ptr(scales))
+    return codes, scales
+
+
+def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact values of unpacked codes with one scale byte per 32 codes (fp64)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    assert codes.size == scales.size * 32
+    out = np.empty(codes.shape, np.float64)
+    lib().mxref_dequantize(_ptr(codes), _ptr(scales), scales.size, _ptr(out))
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# Attention
+# ----------------------------------------------------------------------------------------------
+
+def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=True, rule=RULE_UOS,
+                   qmax=7.25, tau=0.0, weights=False):
+    """Online-softmax attention with PNQ for query rows qd [n, d] against
+    kd, vd [N, d] (fp64 values).  Returns dict(out, m, l[, wsum, ocheck])."""
+    qd = np.ascontiguousarray(qd, dtype=np.float64)
+    kd = np.ascontiguousarray(kd, dtype=np.float64)
+    vd = np.ascontiguousarray(vd, dtype=np.float64)
+    n, d = qd.shape
+    N = kd.shape[0]
+    assert kd.shape == (N, d) and vd.shape == (N, d) and key_tile % 32 == 0
+    cfg = AttnCfg(int(key_tile), int(bool(pnq)), int(bool(quant_p)), int(rule), float(qmax), float(tau))
+    out = np.empty((n, d), np.float64)
+    m = np.empty(n, np.float64)
+    l = np.empty(n, np.float64)
+    wsum = np.empty(n, np.float64) if weights else None
+    ocheck = np.empty((n, d), np.float64) if weights else None
+    lib().mxref_attention_rows(_ptr(qd), n, _ptr(kd), _ptr(vd), N, d, float(np.float32(softmax_scale)),
+                               ctypes.byref(cfg), _ptr(out), _ptr(m), _ptr(l), _ptr(wsum), _ptr(ocheck))
+    res = {"out": out, "m": m, "l": l}
+    if weights:
+        res["wsum"] = wsum
+        res["ocheck"] = ocheck
+    return res
+
+
+def prepare_head(q, k, v, rotate=True, rule=RULE_UOS, qmax=7.25, quant=True):
+    """Rotate/quantize one head's Q [nq, d], K [N, d], V [N, d] (fp32) and
+    return their exact dequantized values (fp64): Q, K groups along d, V
+    groups of 32 consecutive keys per channel."""
+    q = np.ascontiguousarray(q, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    if not quant:
+        qr = rotate_rows(q) if rotate else q
+        kr = rotate_rows(k) if rotate else k
+        return qr.astype(np.float64), kr.astype(np.float64), v.astype(np.float64)
+    qc, qs = rotate_quantize_rows(q, rotate, rule, qmax)
+    kc, ks = rotate_quantize_rows(k, rotate, rule, qmax)
+    vc, vs = quantize(v, axis=1, rule=rule, qmax=qmax)      # [d, ceil(N/32)*32]
+    N = v.shape[0]
+    vd = dequantize(vc, vs)[:, :N].T                           # [N, d]
+    return dequantize(qc, qs), dequantize(kc, ks), np.ascontiguousarray(vd)
+
+
+def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=7.25, pnq=True,
+                 key_tile=64, tau=0.0, quant=True, weights=False):
+    """MXAttention forward for selected query rows of every head.
+
+    q, k, v: fp32 arrays [BH, N, d] (exact upcasts of the inputs).
+    rows:    int array of query indices (same rows for every head).
+    Returns dict with out [BH, len(rows), d] (fp64) and m, l [BH, len(rows)].
+    """
+    BH, N, d = q.shape
+    rows = np.asarray(rows, dtype=np.int64)
+    outs, ms, ls, ws, ocs = [], [], [], [], []
+    for h in range(BH):
+        qd, kd, vd = prepare_head(q[h][rows], k[h], v[h], rotate, rule, qmax, quant)
+        r = attention_rows(qd, kd, vd, softmax_scale, key_tile, pnq, quant, rule, qmax, tau, weights)
+        outs.append(r["out"])
+        ms.append(r["m"])
+        ls.append(r["l"])
+        if weights:
+            ws.append(r["wsum"])
+            ocs.append(r["ocheck"])
+    res = {"out": np.stack(outs), "m": np.stack(ms), "l": np.stack(ls)}
+    if weights:
+        res["wsum"] = np.stack(ws)
+        res["ocheck"] = np.stack(ocs)
+    return res
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to fp32 and then to bf16 (round to nearest, ties to
+    even), returned as fp64 values; finite inputs only."""
+    f = np.asarray(x, dtype=np.float32)
+    b = f.view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    r = ((b + 0x7FFF + lsb) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)

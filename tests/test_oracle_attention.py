@@ -1,0 +1,104 @@
+"""Pins of the oracle's online-softmax attention with PNQ: the textbook case
+with quantization off, Proposition 1 (induced weights sum to one), the output
+rebuilt from those weights, a hand-computed PNQ example and closed-form
+special cases."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from conftest import golden
+from mxfp4_bit_attention_b200 import inputs
+
+
+def _softmax_attention(q, k, v, s):
+    S = (q @ k.T) * s
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    return (P / P.sum(axis=1, keepdims=True)) @ v
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    g = inputs.generate("tiny")
+    return [inputs.as_fp32(g[n], "fp32")[0] for n in "qkv"]
+
+
+@pytest.mark.parametrize("rotate", [False, True])
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_quant_off_equals_softmax_attention(tiny, rotate, tau):
+    q, k, v = tiny
+    s = 1 / math.sqrt(q.shape[1])
+    res = oracle.forward_rows(q[None], k[None], v[None], np.arange(q.shape[0]), s, rotate=rotate,
+                              quant=False, key_tile=64, tau=tau)
+    ref = _softmax_attention(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64), s)
+    assert np.max(np.abs(res["out"][0] - ref)) <= 1e-5
+
+
+@pytest.mark.parametrize("rule", [oracle.RULE_UOS, oracle.RULE_QMAX6, oracle.RULE_OCP])
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_pnq_weights_sum_to_one(tiny, rule, tau):
+    q, k, v = tiny
+    qd, kd, vd = oracle.prepare_head(q, k, v, True, rule)
+    r = oracle.attention_rows(qd, kd, vd, 0.125, 64, pnq=True, rule=rule, tau=tau, weights=True)
+    assert np.max(np.abs(r["wsum"] - 1.0)) <= 1e-12
+    assert np.max(np.abs(r["ocheck"] - r["out"])) <= 1e-12
+
+
+def test_direct_placement_breaks_normalization(tiny):
+    q, k, v = tiny
+    qd, kd, vd = oracle.prepare_head(q, k, v, True, oracle.RULE_OCP)
+    r = oracle.attention_rows(qd, kd, vd, 0.125, 64, pnq=False, rule=oracle.RULE_OCP, weights=True)
+    dev = r["wsum"] - 1.0
+    assert np.mean(np.abs(dev) > 1e-6) > 0.9
+    assert np.max(np.abs(r["ocheck"] - r["out"])) <= 1e-12
+
+
+def test_hand_computed_pnq_example():
+    ex = golden("pnq_example.json")
+    p = np.array(ex["p"])
+    n = len(p)
+    d = 8
+    q = np.zeros((1, d)); q[0, 0] = 1.0
+    k = np.zeros((n, d)); k[:, 0] = np.log(p).astype(np.float32)
+    v = np.eye(n, d)
+    for rule in (oracle.RULE_UOS, oracle.RULE_QMAX6, oracle.RULE_OCP):
+        r = oracle.attention_rows(q, k, v, 1.0, 32, pnq=True, rule=rule, weights=True)
+        assert np.allclose(r["out"][0], ex["out_pnq"], rtol=0, atol=1e-15)
+        assert r["l"][0] == pytest.approx(ex["l_pnq"], abs=1e-15)
+        assert r["wsum"][0] == pytest.approx(ex["wsum_pnq"], abs=1e-15)
+        rd = oracle.attention_rows(q, k, v, 1.0, 32, pnq=False, rule=rule, weights=True)
+        assert rd["l"][0] == pytest.approx(ex["l_direct"], rel=1e-6)
+        assert np.allclose(rd["out"][0], np.array(ex["p_hat"]) / ex["l_direct"], rtol=1e-6)
+        assert rd["wsum"][0] == pytest.approx(ex["wsum_direct"], rel=1e-6)
+
+
+def test_equal_scores_give_mean_of_values():
+    """All keys equal: every P~ is exp(0) = 1, which MXFP4 represents exactly,
+    so l = N and O is the plain mean of V over N keys (ragged last tile)."""
+    rng = np.random.default_rng(3)
+    N, d = 150, 64
+    q = rng.standard_normal((4, d))
+    k = np.tile(rng.standard_normal((1, d)), (N, 1))
+    v = rng.standard_normal((N, d))
+    r = oracle.attention_rows(q, k, v, 0.125, 64, pnq=True)
+    assert np.allclose(r["l"], N, rtol=0, atol=1e-12)
+    assert np.allclose(r["out"], v.mean(axis=0)[None], rtol=0, atol=1e-12)
+
+
+def test_single_dominant_key():
+    """One key far above the rest: P~ underflows to zero elsewhere, O = v of that key."""
+    N, d = 100, 32
+    q = np.zeros((1, d)); q[0, 0] = 1
+    k = np.zeros((N, d)); k[:, 0] = -200.0; k[37, 0] = 0.0
+    v = np.arange(N * d, dtype=np.float64).reshape(N, d)
+    r = oracle.attention_rows(q, k, v, 1.0, 64, pnq=True)
+    assert np.array_equal(r["out"][0], v[37])
+
+
+def test_rows_are_independent(tiny):
+    q, k, v = tiny
+    rows = np.array([0, 5, 200, 255])
+    full = oracle.forward_rows(q[None], k[None], v[None], np.arange(256), 0.125)
+    part = oracle.forward_rows(q[None], k[None], v[None], rows, 0.125)
+    assert np.array_equal(full["out"][0][rows], part["out"][0])
