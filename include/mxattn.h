@@ -77,6 +77,12 @@ extern "C" {
 
 #define MXATTN_ABI_VERSION 1
 
+#if defined(__GNUC__)
+#define MXATTN_API __attribute__((visibility("default")))
+#else
+#define MXATTN_API
+#endif
+
 typedef enum mxattn_status {
   MXATTN_OK = 0,
   MXATTN_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad option value        */
@@ -90,7 +96,7 @@ typedef enum mxattn_scale_rule {
   MXATTN_SCALE_UOS = 0,        /* ceiling rule, boundary 29/4: max -> (3.625, 7.25] */
   MXATTN_SCALE_QMAX6 = 1,      /* ceiling rule, boundary 6:    max -> (3, 6]        */
   MXATTN_SCALE_OCP = 2,        /* OCP floor rule e = floor(log2 amax) - 2: [4, 8)  */
-  MXATTN_SCALE_CEIL_CUSTOM = 3 /* ceiling rule, boundary opts.qmax (> 0, finite)   */
+  MXATTN_SCALE_CEIL_CUSTOM = 3 /* ceiling rule, boundary opts.qmax in [4, 8]       */
 } mxattn_scale_rule;
 
 typedef enum mxattn_dtype { MXATTN_BF16 = 0, MXATTN_FP32 = 1 } mxattn_dtype;
@@ -110,20 +116,20 @@ typedef struct mxattn_opts {
 
 /* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
  * key_tile 64, rescale_tau 8, no workspace. */
-void mxattn_opts_default(mxattn_opts* opts);
+MXATTN_API void mxattn_opts_default(mxattn_opts* opts);
 
 /* Bytes of workspace mxattn_forward needs for this problem (status block plus
  * packed Q, K, V operands); 0 for invalid sizes. */
-size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts);
+MXATTN_API size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts);
 
 /* Sizes of the packed attention operands described above (0 for invalid sizes). */
-size_t mxattn_qk_codes_bytes(int B, int H, int N, int d);
-size_t mxattn_qk_scales_bytes(int B, int H, int N, int d);
-size_t mxattn_v_codes_bytes(int B, int H, int N, int d);
-size_t mxattn_v_scales_bytes(int B, int H, int N, int d);
+MXATTN_API size_t mxattn_qk_codes_bytes(int B, int H, int N, int d);
+MXATTN_API size_t mxattn_qk_scales_bytes(int B, int H, int N, int d);
+MXATTN_API size_t mxattn_v_codes_bytes(int B, int H, int N, int d);
+MXATTN_API size_t mxattn_v_scales_bytes(int B, int H, int N, int d);
 
 /* Zero the workspace status block (enqueued on stream). */
-mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* stream);
+MXATTN_API mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* stream);
 
 /*
  * Generic MXFP4 quantization of a row-major [rows][cols] matrix x
@@ -136,7 +142,7 @@ mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* stream);
  *                scales [cols][ceil(rows/32)].
  * Partial tail groups are zero-padded.  No rotation is applied.
  */
-mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, int group_axis,
+MXATTN_API mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, int group_axis,
                                     const mxattn_opts* opts, uint8_t* codes, uint8_t* scales,
                                     void* stream);
 
@@ -149,7 +155,7 @@ mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, i
  * fl32(1/sqrt(d)); the scale rule reads these fp32 values.
  * d in {64, 128}.  Buffers: mxattn_qk_codes_bytes / mxattn_qk_scales_bytes.
  */
-mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
+MXATTN_API mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
                                        const mxattn_opts* opts, uint8_t* q_codes,
                                        uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales,
                                        void* stream);
@@ -158,7 +164,7 @@ mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int 
  * Step 2 for V: MXFP4 quantization in groups of 32 consecutive keys per
  * channel (no rotation), written in the packed V operand layout.
  */
-mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mxattn_opts* opts,
+MXATTN_API mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mxattn_opts* opts,
                              uint8_t* v_codes, uint8_t* v_scales, void* stream);
 
 /*
@@ -169,7 +175,7 @@ mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mx
  * (PNQ) or from the unquantized one (pnq = 0), O~ += P^ V^, O = O~ / l in
  * opts->dtype.  Requires opts->workspace (status block, >= 256 bytes).
  */
-mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
+MXATTN_API mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales,
                                      const uint8_t* k_codes, const uint8_t* k_scales,
                                      const uint8_t* v_codes, const uint8_t* v_scales, int B, int H,
                                      int N, int d, float softmax_scale, const mxattn_opts* opts,
@@ -179,7 +185,7 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
  * The whole forward pass: mxattn_hadamard_quant_qk + mxattn_quant_v into
  * the workspace, then mxattn_attention_mxfp4.  d in {64, 128}, N >= 1.
  */
-mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B, int H, int N,
+MXATTN_API mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B, int H, int N,
                              int d, float softmax_scale, const mxattn_opts* opts, void* out,
                              void* stream);
 
@@ -188,10 +194,10 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
  * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
  * last call (its output is then undefined), MXATTN_OK otherwise.
  */
-mxattn_status mxattn_get_device_error(const mxattn_opts* opts, void* stream);
+MXATTN_API mxattn_status mxattn_get_device_error(const mxattn_opts* opts, void* stream);
 
 /* Static string naming a status code. */
-const char* mxattn_status_string(mxattn_status status);
+MXATTN_API const char* mxattn_status_string(mxattn_status status);
 
 /*
  * Dense FP4 tensor-core throughput probe (not part of the method): `ctas`
@@ -200,7 +206,7 @@ const char* mxattn_status_string(mxattn_status status);
  * n in {64, 128, 256}.  The caller times the launch; flops = ctas * iters *
  * 2 * 128 * n * 64.
  */
-mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream);
+MXATTN_API mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream);
 
 #ifdef __cplusplus
 }

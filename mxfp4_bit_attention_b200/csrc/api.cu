@@ -1,0 +1,285 @@
+// api.cu -- the C ABI declared in include/mxattn.h: argument validation, workspace carving and
+// kernel launches.  No allocation, no synchronization (except mxattn_get_device_error).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mxattn.h"
+#include "kernels.cuh"
+
+using namespace mxattn;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr long long kWaitBudgetCycles = 2000000000LL;  // ~1 s at the B200's clocks
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool sizes_ok(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return false;
+  if (d != 64 && d != 128) return false;
+  if ((int64_t)B * H > 65535) return false;  // grid.y of the attention launch
+  return true;
+}
+
+int64_t t128(int N) { return ((int64_t)N + 127) / 128; }
+int64_t t64(int N) { return ((int64_t)N + 63) / 64; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Boundary q = mq * 2^eq of a ceiling rule, or the OCP floor rule.
+bool make_rule(const mxattn_opts* o, ScaleRule* r) {
+  float q;
+  switch (o->scale_rule) {
+    case MXATTN_SCALE_UOS: q = 7.25f; break;
+    case MXATTN_SCALE_QMAX6: q = 6.0f; break;
+    case MXATTN_SCALE_OCP: r->eq = 2; r->mq = 0xFFFFFFFFu; return true;
+    case MXATTN_SCALE_CEIL_CUSTOM:
+      q = o->qmax;
+      if (!(q >= 4.0f && q <= 8.0f)) return false;  // keeps every exponent inside [-127, 126]
+      break;
+    default: return false;
+  }
+  uint32_t bits;
+  std::memcpy(&bits, &q, 4);
+  r->eq = (int)(bits >> 23) - 127;
+  r->mq = bits & 0x007FFFFFu;
+  return true;
+}
+
+mxattn_status check_opts(const mxattn_opts* o) {
+  if (o == nullptr) return MXATTN_ERR_INVALID_ARG;
+  ScaleRule r;
+  if (!make_rule(o, &r)) return MXATTN_ERR_INVALID_ARG;
+  if (o->dtype != MXATTN_BF16 && o->dtype != MXATTN_FP32) return MXATTN_ERR_INVALID_ARG;
+  if (o->pnq != 0 && o->pnq != 1) return MXATTN_ERR_INVALID_ARG;
+  if (o->rotate != 0 && o->rotate != 1) return MXATTN_ERR_INVALID_ARG;
+  if (!(o->rescale_tau >= 0.f && std::isfinite(o->rescale_tau))) return MXATTN_ERR_INVALID_ARG;
+  if (o->key_tile != 64) return o->key_tile == 128 ? MXATTN_ERR_UNSUPPORTED : MXATTN_ERR_INVALID_ARG;
+  return MXATTN_OK;
+}
+
+struct Carve {
+  size_t q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, total;
+};
+
+Carve carve(int B, int H, int N, int d) {
+  Carve c;
+  size_t off = kStatusBytes;
+  c.q_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, N, d));
+  c.q_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, N, d));
+  c.k_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, N, d));
+  c.k_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, N, d));
+  c.v_codes = off; off = align256(off + mxattn_v_codes_bytes(B, H, N, d));
+  c.v_scales = off; off = align256(off + mxattn_v_scales_bytes(B, H, N, d));
+  c.total = off;
+  return c;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+mxattn_status launched(cudaError_t e) { return e == cudaSuccess ? MXATTN_OK : MXATTN_ERR_CUDA; }
+
+mxattn_status check_workspace(const mxattn_opts* o, size_t need) {
+  if (o->workspace == nullptr || o->workspace_bytes < need) return MXATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(o->workspace) & 255u) != 0) return MXATTN_ERR_WORKSPACE;
+  return MXATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void mxattn_opts_default(mxattn_opts* o) {
+  if (o == nullptr) return;
+  o->scale_rule = MXATTN_SCALE_UOS;
+  o->qmax = 7.25f;
+  o->pnq = 1;
+  o->rotate = 1;
+  o->dtype = MXATTN_BF16;
+  o->key_tile = 64;
+  o->rescale_tau = 8.0f;
+  o->workspace = nullptr;
+  o->workspace_bytes = 0;
+}
+
+size_t mxattn_qk_codes_bytes(int B, int H, int N, int d) {
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return (size_t)B * H * t128(N) * 128 * (d / 2);
+}
+size_t mxattn_qk_scales_bytes(int B, int H, int N, int d) {
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return (size_t)B * H * t128(N) * 512;
+}
+size_t mxattn_v_codes_bytes(int B, int H, int N, int d) {
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return (size_t)B * H * t64(N) * d * 32;
+}
+size_t mxattn_v_scales_bytes(int B, int H, int N, int d) {
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return (size_t)B * H * t128(N) * 512;
+}
+
+size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts) {
+  (void)opts;
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return carve(B, H, N, d).total;
+}
+
+mxattn_status mxattn_workspace_init(const mxattn_opts* o, void* stream) {
+  if (o == nullptr) return MXATTN_ERR_INVALID_ARG;
+  if (check_workspace(o, kStatusBytes) != MXATTN_OK) return MXATTN_ERR_WORKSPACE;
+  return launched(cudaMemsetAsync(o->workspace, 0, kStatusBytes, as_stream(stream)));
+}
+
+mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, int group_axis,
+                                    const mxattn_opts* o, uint8_t* codes, uint8_t* scales, void* stream) {
+  if (x == nullptr || codes == nullptr || scales == nullptr || rows < 1 || cols < 1) return MXATTN_ERR_INVALID_ARG;
+  if (group_axis != 0 && group_axis != 1) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(codes)) return MXATTN_ERR_INVALID_ARG;
+  const int64_t outer = group_axis == 0 ? rows : cols;
+  const int64_t inner = group_axis == 0 ? cols : rows;
+  if (outer * ((inner + 31) / 32) > ((int64_t)1 << 38)) return MXATTN_ERR_UNSUPPORTED;
+  PlainQuantArgs a;
+  a.x = x;
+  a.codes = codes;
+  a.scales = scales;
+  a.rows = rows;
+  a.cols = cols;
+  a.axis = group_axis;
+  make_rule(o, &a.rule);
+  return launched(launch_quant_plain(a, o->dtype, as_stream(stream)));
+}
+
+mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
+                                       const mxattn_opts* o, uint8_t* q_codes, uint8_t* q_scales,
+                                       uint8_t* k_codes, uint8_t* k_scales, void* stream) {
+  if (!sizes_ok(B, H, N, d)) return (B >= 1 && H >= 1 && N >= 1 && (d == 64 || d == 128)) ? MXATTN_ERR_UNSUPPORTED
+                                                                                          : MXATTN_ERR_INVALID_ARG;
+  if (!q || !k || !q_codes || !q_scales || !k_codes || !k_scales) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes)) return MXATTN_ERR_INVALID_ARG;
+  QKQuantArgs a;
+  a.q = q;
+  a.k = k;
+  a.q_codes = q_codes;
+  a.q_scales = q_scales;
+  a.k_codes = k_codes;
+  a.k_scales = k_scales;
+  a.BH = B * H;
+  a.N = N;
+  a.rotate = o->rotate;
+  a.hadamard_scale = (float)(1.0 / std::sqrt((double)d));
+  make_rule(o, &a.rule);
+  return launched(launch_rotate_quant_qk(a, d, o->dtype, as_stream(stream)));
+}
+
+mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mxattn_opts* o, uint8_t* v_codes,
+                             uint8_t* v_scales, void* stream) {
+  if (!sizes_ok(B, H, N, d)) return MXATTN_ERR_INVALID_ARG;
+  if (!v || !v_codes || !v_scales) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(v) || !aligned16(v_codes)) return MXATTN_ERR_INVALID_ARG;
+  VQuantArgs a;
+  a.v = v;
+  a.v_codes = v_codes;
+  a.v_scales = v_scales;
+  a.BH = B * H;
+  a.N = N;
+  make_rule(o, &a.rule);
+  return launched(launch_quant_v(a, d, o->dtype, as_stream(stream)));
+}
+
+mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                     const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales,
+                                     int B, int H, int N, int d, float softmax_scale, const mxattn_opts* o,
+                                     void* out, void* stream) {
+  if (!sizes_ok(B, H, N, d)) return MXATTN_ERR_INVALID_ARG;
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !v_codes || !v_scales || !out) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  st = check_workspace(o, kStatusBytes);
+  if (st != MXATTN_OK) return st;
+  const void* ptrs[] = {q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MXATTN_ERR_INVALID_ARG;
+  AttnArgs a;
+  a.q_codes = q_codes;
+  a.q_scales = q_scales;
+  a.k_codes = k_codes;
+  a.k_scales = k_scales;
+  a.v_codes = v_codes;
+  a.v_scales = v_scales;
+  a.out = out;
+  a.status = reinterpret_cast<int*>(o->workspace);
+  a.BH = B * H;
+  a.N = N;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+  a.tau = o->rescale_tau;
+  a.pnq = o->pnq;
+  make_rule(o, &a.rule);
+  a.wait_budget = kWaitBudgetCycles;
+  return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
+}
+
+mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                             float softmax_scale, const mxattn_opts* o, void* out, void* stream) {
+  if (!sizes_ok(B, H, N, d)) return MXATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  const Carve c = carve(B, H, N, d);
+  st = check_workspace(o, c.total);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
+  st = mxattn_hadamard_quant_qk(q, k, B, H, N, d, o, ws + c.q_codes, ws + c.q_scales, ws + c.k_codes,
+                                ws + c.k_scales, stream);
+  if (st != MXATTN_OK) return st;
+  st = mxattn_quant_v(v, B, H, N, d, o, ws + c.v_codes, ws + c.v_scales, stream);
+  if (st != MXATTN_OK) return st;
+  return mxattn_attention_mxfp4(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes,
+                                ws + c.v_scales, B, H, N, d, softmax_scale, o, out, stream);
+}
+
+mxattn_status mxattn_get_device_error(const mxattn_opts* o, void* stream) {
+  if (o == nullptr) return MXATTN_ERR_INVALID_ARG;
+  if (check_workspace(o, kStatusBytes) != MXATTN_OK) return MXATTN_ERR_WORKSPACE;
+  int words[4] = {0, 0, 0, 0};
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemcpyAsync(words, o->workspace, sizeof(words), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MXATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (words[0] == 0) return MXATTN_OK;
+  if (cudaMemsetAsync(o->workspace, 0, kStatusBytes, s) != cudaSuccess) return MXATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MXATTN_ERR_CUDA;
+  return MXATTN_ERR_TIMEOUT;
+}
+
+const char* mxattn_status_string(mxattn_status s) {
+  switch (s) {
+    case MXATTN_OK: return "MXATTN_OK";
+    case MXATTN_ERR_INVALID_ARG: return "MXATTN_ERR_INVALID_ARG";
+    case MXATTN_ERR_UNSUPPORTED: return "MXATTN_ERR_UNSUPPORTED";
+    case MXATTN_ERR_WORKSPACE: return "MXATTN_ERR_WORKSPACE";
+    case MXATTN_ERR_CUDA: return "MXATTN_ERR_CUDA";
+    case MXATTN_ERR_TIMEOUT: return "MXATTN_ERR_TIMEOUT";
+  }
+  return "unknown mxattn_status";
+}
+
+mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream) {
+  if (ctas < 1 || ctas > 65535 || iters < 1 || (n != 64 && n != 128 && n != 256)) return MXATTN_ERR_INVALID_ARG;
+  return launched(launch_fp4_mma_probe(ctas, iters, n, nullptr, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,384 @@
+// attn.cu -- fused MXFP4 attention with Pre-Normalization Quantization on tcgen05.
+//
+// Method: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for
+// MXFP4 Attention" -- Pith review page, Fig. 4 (FlashAttention loop; PNQ quantizes the
+// unnormalized exponential tile once and feeds the same quantized tile to the row sum l and
+// to the output update; direct placement uses the unquantized tile for l) and Fig. 1 (UOS
+// scaling for every MXFP4 tensor in attention); 10100.com article (same mechanism).
+//
+// One CTA owns 128 query rows of one head and sweeps all keys in tiles of 64:
+//   warp 4 (one lane)  bulk-copies Q^ once and K^/V^ tiles + their scale atoms into a
+//                      4-stage shared-memory ring;
+//   warp 5 (one lane)  issues tcgen05.mma kind::mxf4 block-scaled MMAs:
+//                      S = Q^ K^T (TMEM, fp32) and O~ += P^ V^ (TMEM, fp32);
+//   warps 0-3          one query row per thread: read S from TMEM, online max (optionally lazy,
+//                      threshold tau in log2 units), P~ = 2^(S*c - m) folded with the MXFP4 scale
+//                      of each 32-key group, E2M1 codes of P~ written to shared memory in the
+//                      MMA operand layout, group scales written as a scale atom, l updated from
+//                      the quantized codes (PNQ) or from P~ (direct placement), O~ rescaled in
+//                      TMEM when the running max moves, and finally O = O~ / l.
+// Two CTAs share an SM (256 TMEM columns each), so one CTA's softmax overlaps the other's MMAs.
+// Every wait is bounded; on expiry the CTA records a status word, drains its in-flight copies
+// and MMAs, frees its TMEM and exits.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mxattn {
+
+constexpr int kBM = 128;      // query rows per CTA
+constexpr int kBN = 64;       // keys per tile
+constexpr int kStages = 4;    // K/V ring depth
+constexpr int kThreads = 192; // 4 softmax warps, producer warp, MMA warp
+constexpr uint32_t kTmemCols = 256;
+
+template <int D>
+struct Layout {
+  // shared memory, byte offsets from a 1024-byte aligned base
+  static constexpr int Q_BYTES = kBM * D / 2;
+  static constexpr int K_BYTES = kBN * D / 2;
+  static constexpr int V_BYTES = D * kBN / 2;
+  static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+  static constexpr int Q_CODES = 0;
+  static constexpr int STAGE0 = Q_BYTES;
+  static constexpr int P_CODES = STAGE0 + kStages * STAGE_BYTES;
+  static constexpr int P_BYTES = kBM * kBN / 2;
+  static constexpr int SF_Q = P_CODES + P_BYTES;
+  static constexpr int SF_P = SF_Q + 512;
+  static constexpr int SF_K = SF_P + 512;
+  static constexpr int SF_V = SF_K + kStages * 512;
+  static constexpr int BARS = SF_V + kStages * 512;
+  enum {
+    B_Q = 0,
+    B_KV_FULL = 1,
+    B_KV_EMPTY = 1 + kStages,
+    B_S_FULL = 1 + 2 * kStages,
+    B_S_FREE,
+    B_P_FULL,
+    B_O_DONE,
+    B_DRAIN,
+    NUM_BARS
+  };
+  static constexpr int TMEM_SLOT = BARS + NUM_BARS * 8;
+  static constexpr int ABORT = TMEM_SLOT + 4;
+  static constexpr int TOTAL = ABORT + 4;
+  // slack for aligning the base; at least 80 KB so that no third CTA (which would block in
+  // tcgen05.alloc until a neighbour frees its columns) becomes resident on an SM
+  static constexpr int DYN_SMEM = TOTAL + 1024 > 80 * 1024 ? TOTAL + 1024 : 80 * 1024;
+  // tensor memory columns
+  static constexpr uint32_t T_S = 0;
+  static constexpr uint32_t T_O = 64;
+  static constexpr uint32_t T_SFQ = 64 + D;
+  static constexpr uint32_t T_SFP = T_SFQ + 4;
+  static constexpr uint32_t T_SFK = T_SFP + 4;
+  static constexpr uint32_t T_SFV = T_SFK + 4 * kStages;
+  static_assert(T_SFV + 4 * kStages <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t QK_LAYOUT = D == 128 ? kLayoutSW64 : kLayoutSW32;
+};
+
+__device__ __forceinline__ void raise_abort(volatile int* flag, int* status, int where) {
+  *flag = 1;
+  if (atomicCAS(status, 0, kStatusTimeout) == 0) atomicExch(status + 1, where);
+}
+
+template <int D, int DT, bool PNQ>
+__global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T128 = (a.N + 127) / 128;
+  const int T64 = (a.N + 63) / 64;
+  const int qt = blockIdx.x;
+  const int bh = blockIdx.y;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::ABORT);
+  __shared__ int never;  // a flag nothing sets: drains ignore the abort flag
+  auto bar = [&](int i) -> uint32_t { return sb + L::BARS + 8 * i; };
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    never = 0;
+    mbar_init(bar(L::B_Q), 1);
+    for (int s = 0; s < kStages; s++) {
+      mbar_init(bar(L::B_KV_FULL + s), 1);
+      mbar_init(bar(L::B_KV_EMPTY + s), 1);
+    }
+    mbar_init(bar(L::B_S_FULL), 1);
+    mbar_init(bar(L::B_S_FREE), 4);
+    mbar_init(bar(L::B_P_FULL), 4);
+    mbar_init(bar(L::B_O_DONE), 1);
+    mbar_init(bar(L::B_DRAIN), 1);
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TMEM_SLOT);
+  const volatile int* no_abort = &never;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      const size_t qtile = (size_t)bh * T128 + qt;
+      mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES + 512);
+      bulk_g2s(sb + L::Q_CODES, a.q_codes + qtile * (size_t)L::Q_BYTES, L::Q_BYTES, bar(L::B_Q));
+      bulk_g2s(sb + L::SF_Q, a.q_scales + qtile * 512, 512, bar(L::B_Q));
+      for (int j = 0; j < T64; j++) {
+        const int s = j % kStages;
+        if (j >= kStages) {
+          ok = mbar_wait(bar(L::B_KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, a.wait_budget);
+          if (!ok) break;
+        }
+        const uint32_t fb = bar(L::B_KV_FULL + s);
+        const size_t t128 = (size_t)bh * T128 + j / 2;
+        mbar_arrive_expect_tx(fb, L::K_BYTES + L::V_BYTES + 1024);
+        bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES,
+                 a.k_codes + (t128 * kBM + (j % 2) * kBN) * (size_t)(D / 2), L::K_BYTES, fb);
+        bulk_g2s(sb + L::SF_K + s * 512, a.k_scales + t128 * 512, 512, fb);
+        bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES + L::K_BYTES,
+                 a.v_codes + ((size_t)bh * T64 + j) * (size_t)L::V_BYTES, L::V_BYTES, fb);
+        bulk_g2s(sb + L::SF_V + s * 512, a.v_scales + t128 * 512, 512, fb);
+        issued = j + 1;
+      }
+      if (!ok) {
+        raise_abort(abort_flag, a.status, 1);
+        // let every copy already issued land before the CTA can exit
+        mbar_wait(bar(L::B_Q), 0, no_abort, a.wait_budget);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; j++)
+          mbar_wait(bar(L::B_KV_FULL + j % kStages), (j / kStages) & 1, no_abort, a.wait_budget);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget);
+      if (ok) {
+        tc_fence_after();
+        tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
+        const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
+        const uint64_t pdesc = smem_desc(sb + L::P_CODES, 16, 8 * (kBN / 2), kLayoutSW32);
+        for (int j = 0; j <= T64; j++) {
+          if (j < T64) {
+            const int s = j % kStages;
+            ok = mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget);
+            if (!ok) break;
+            tc_fence_after();
+            tmem_cp_sf_atom(tmem + L::T_SFK + 4 * s, sb + L::SF_K + 512 * s);
+            tmem_cp_sf_atom(tmem + L::T_SFV + 4 * s, sb + L::SF_V + 512 * s);
+            if (j > 0) {
+              ok = mbar_wait(bar(L::B_S_FREE), (j - 1) & 1, abort_flag, a.wait_budget);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint64_t kdesc = smem_desc(sb + L::STAGE0 + s * L::STAGE_BYTES, 16, 8 * (D / 2), L::QK_LAYOUT);
+#pragma unroll
+            for (int kb = 0; kb < D / 64; kb++) {
+              // K block kb covers head dims 64kb..64kb+63: 32 bytes further along each row,
+              // scale bytes 2kb and 2kb+1 of each row's scale word.
+              mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
+                       mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
+                       tmem + L::T_SFK + 4 * s + 2 * (j & 1), kb > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(L::B_S_FULL));
+          }
+          if (j > 0) {
+            const int jp = j - 1, sp = jp % kStages;
+            ok = mbar_wait(bar(L::B_P_FULL), jp & 1, abort_flag, a.wait_budget);
+            if (!ok) break;
+            tc_fence_after();
+            tmem_cp_sf_atom(tmem + L::T_SFP, sb + L::SF_P);
+            const uint64_t vdesc =
+                smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
+            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, D, 0, 2 * (jp & 1)), tmem + L::T_SFP,
+                     tmem + L::T_SFV + 4 * sp, jp > 0 ? 1u : 0u);
+            mma_commit(bar(L::B_O_DONE));
+            mma_commit(bar(L::B_KV_EMPTY + sp));
+          }
+        }
+      }
+      if (!ok) raise_abort(abort_flag, a.status, 2);
+      // wait for every tcgen05 operation this thread issued before TMEM is released
+      mma_commit(bar(L::B_DRAIN));
+      mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax (warps 0-3)
+    const int row = threadIdx.x;  // TMEM lane and query row within the tile
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const float c = a.scale_log2;
+    float m2 = -INFINITY;  // running max of S*c (log2 units) actually used for the exponent
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T64; j++) {
+      ok = mbar_wait(bar(L::B_S_FULL), j & 1, abort_flag, a.wait_budget);
+      if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s0[32], s1[32];
+      tmem_ld32(tl + L::T_S, s0);
+      tmem_ld32(tl + L::T_S + 32, s1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_S_FREE));
+
+      const int valid = min(kBN, a.N - j * kBN);
+      float gmax[2];
+#pragma unroll
+      for (int g = 0; g < 2; g++) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          const float s = __uint_as_float(g == 0 ? s0[i] : s1[i]);
+          mx = fmaxf(mx, (g * 32 + i < valid) ? s : -INFINITY);
+        }
+        gmax[g] = mx;
+      }
+      const float mt = fmaxf(gmax[0], gmax[1]) * c;
+      const bool first = (j == 0);
+      const bool move = first || (mt > m2 + a.tau);
+      const float mnew = move ? mt : m2;
+      const float alpha = first ? 0.f : (move ? ex2_approx(m2 - mnew) : 1.f);
+      m2 = mnew;
+
+      int e[2];
+      float bias[2];
+#pragma unroll
+      for (int g = 0; g < 2; g++) {
+        const float amax = gmax[g] == -INFINITY ? 0.f : ex2_approx(fmaf(gmax[g], c, -m2));
+        e[g] = shared_exponent(amax, a.rule);
+        bias[g] = m2 + (float)e[g];
+      }
+      uint32_t w[8];
+      float psum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 8; q++) {
+        const int g = q / 4;
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+          const int idx = q * 8 + i;
+          const float x = fmaf(__uint_as_float(g == 0 ? s0[idx] : s1[idx - 32]), c, -bias[g]);
+          p[i] = idx < valid ? ex2_approx(x) : 0.f;
+          if (!PNQ) psum[g] += p[i];
+        }
+        w[q] = cvt_e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int g = 0; g < 2; g++) {
+        const float sc = e[g] > -127 ? __uint_as_float((uint32_t)(e[g] + 127) << 23) : 0.f;
+        const float gs = PNQ ? e2m1x32_sum(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]) : psum[g];
+        lsum += gs * sc;
+      }
+      l = alpha * l + lsum;
+
+      if (j > 0) {
+        // PV of the previous tile must be done before P is overwritten or O rescaled
+        ok = mbar_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.wait_budget);
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xFFFFFFFFu, move)) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; cc++) {
+            uint32_t o[32];
+            tmem_ld32(tl + L::T_O + 32 * cc, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tl + L::T_O + 32 * cc, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint8_t* prow = smem + L::P_CODES + row * (kBN / 2);
+      const int sw = (row >> 2) & 1;
+      *reinterpret_cast<uint4*>(prow + (sw * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(prow + ((1 ^ sw) * 16)) = make_uint4(w[4], w[5], w[6], w[7]);
+      *reinterpret_cast<uint16_t*>(smem + L::SF_P + (row % 32) * 16 + (row / 32) * 4) =
+          (uint16_t)((e[0] + 127) | ((e[1] + 127) << 8));
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_P_FULL));
+    }
+    if (ok) {
+      ok = mbar_wait(bar(L::B_O_DONE), (T64 - 1) & 1, abort_flag, a.wait_budget);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const int qrow = qt * kBM + row;
+      const bool store = qrow < a.N;
+      const size_t obase = ((size_t)bh * a.N + (store ? qrow : 0)) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; cc++) {
+        uint32_t o[32];
+        tmem_ld32(tl + L::T_O + 32 * cc, o);
+        tmem_wait_ld();
+        if (store) {
+          if (DT == kBF16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + obase + 32 * cc);
+#pragma unroll
+            for (int v = 0; v < 4; v++) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; i++) {
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[v * 8 + 2 * i]) * inv_l,
+                                                                __uint_as_float(o[v * 8 + 2 * i + 1]) * inv_l);
+                pk[i] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + obase + 32 * cc);
+#pragma unroll
+            for (int v = 0; v < 8; v++)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                   __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+          }
+        }
+      }
+    }
+    if (!ok) raise_abort(abort_flag, a.status, 3);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, int DT, bool PNQ>
+static cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
+  using L = Layout<D>;
+  auto kern = mxattn_fwd_kernel<D, DT, PNQ>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_SMEM);
+  if (err != cudaSuccess) return err;
+  dim3 grid((unsigned)((a.N + kBM - 1) / kBM), (unsigned)a.BH);
+  kern<<<grid, kThreads, L::DYN_SMEM, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s) {
+  if (a.pnq) {
+    if (D == 128) return dtype == kBF16 ? launch_attention_t<128, kBF16, true>(a, s) : launch_attention_t<128, kFP32, true>(a, s);
+    return dtype == kBF16 ? launch_attention_t<64, kBF16, true>(a, s) : launch_attention_t<64, kFP32, true>(a, s);
+  }
+  if (D == 128) return dtype == kBF16 ? launch_attention_t<128, kBF16, false>(a, s) : launch_attention_t<128, kFP32, false>(a, s);
+  return dtype == kBF16 ? launch_attention_t<64, kBF16, false>(a, s) : launch_attention_t<64, kFP32, false>(a, s);
+}
+
+}  // namespace mxattn

@@ -1,0 +1,277 @@
+// ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the kernels use:
+// mbarriers, bulk async copies, tcgen05 (TMEM alloc, block-scaled MMA, commit,
+// smem->TMEM copy, TMEM loads/stores, fences) and the E2M1 conversions.
+#pragma once
+#include <cstdint>
+
+namespace mxattn {
+
+// ------------------------------------------------------------------------------------------------
+// Addresses
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// ------------------------------------------------------------------------------------------------
+// mbarriers
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait.  Gives up (returns false) after `budget` SM clock cycles, or as
+// soon as *abort becomes non-zero (another warp gave up first).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                          long long budget) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > budget) return false;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Bulk async copy global -> shared, completion counted on an mbarrier (bytes).
+// dst and src 16-byte aligned, bytes a multiple of 16.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------------------
+// tcgen05: tensor memory
+// ------------------------------------------------------------------------------------------------
+// Whole warp: allocate `ncols` TMEM columns, base address written to smem[dst].
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for tcgen05 operands (K-major).
+//   start address >> 4 in bits [0,14), leading byte offset >> 4 in [16,30),
+//   stride byte offset >> 4 in [32,46), descriptor version 1 in [46,48),
+//   layout (swizzle) type in [61,64): 0 none, 4 = 64-byte, 6 = 32-byte swizzle.
+enum : uint32_t { kLayoutNone = 0, kLayoutSW64 = 4, kLayoutSW32 = 6 };
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(layout & 7u) << 61;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::mxf4 (block-scaled E2M1 x E2M1 -> f32,
+// UE8M0 scales, both operands K-major, dense, K = 64 per instruction):
+//   b_sf_id [4,6), a_format [7,10) = 1 (E2M1), b_format [10,13) = 1, N>>3 in [17,23),
+//   scale format bit 23 = 1 (UE8M0), M>>4 in [24,29), a_sf_id [29,31).
+__host__ __device__ constexpr uint32_t mxf4_idesc(uint32_t M, uint32_t N, uint32_t a_sf_id,
+                                                  uint32_t b_sf_id) {
+  return ((b_sf_id & 3u) << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | (1u << 23) |
+         ((M >> 4) << 24) | ((a_sf_id & 3u) << 29);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with per-32-element scales from TMEM.  One thread issues.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05 operations of this thread complete.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// Copy a 512-byte scale-factor atom (32 rows x 16 bytes, K-major, no swizzle) from shared
+// memory to 4 TMEM columns, replicated into the 4 lane quadrants.  One thread issues.
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t smem_atom) {
+  const uint64_t desc = smem_desc(smem_atom, 0, 128, kLayoutNone);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+// Warp-collective TMEM loads / stores: lane i of warp w (w = warp index mod 4) touches TMEM lane
+// 32*w + i; 32 consecutive 32-bit columns starting at taddr's column.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------------------------------------------
+// E2M1 conversions and fast exp2
+// ------------------------------------------------------------------------------------------------
+// Four pairs of fp32 -> four bytes of packed E2M1 codes (round to nearest even, saturating).
+// Byte i holds (lo = a[2i], hi = a[2i+1]); element 2i lands in the low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3, float a4, float a5,
+                                               float a6, float a7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+  return out;
+}
+
+// Sum of the eight E2M1 values packed in a 32-bit word, as an f16x2 pair of partial sums.
+// Exact: every partial sum is a multiple of 0.5 below 64.
+__device__ __forceinline__ uint32_t e2m1x8_sum_h2(uint32_t w) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+      "add.rn.f16x2 h0, h0, h1;\n\t"
+      "add.rn.f16x2 h2, h2, h3;\n\t"
+      "add.rn.f16x2 %0, h0, h2;\n\t}"
+      : "=r"(out)
+      : "r"(w));
+  return out;
+}
+
+// Sum of the 32 E2M1 values packed in four words, as fp32 (exact: at most 32 * 6 = 192, a
+// multiple of 0.5, so every f16 partial sum is exact).
+__device__ __forceinline__ float e2m1x32_sum(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  float out;
+  asm("{\n\t.reg .b32 a, b, c, d;\n\t.reg .b16 lo, hi;\n\t.reg .f32 flo, fhi;\n\t"
+      "add.rn.f16x2 a, %1, %2;\n\t"
+      "add.rn.f16x2 b, %3, %4;\n\t"
+      "add.rn.f16x2 c, a, b;\n\t"
+      "mov.b32 {lo, hi}, c;\n\t"
+      "cvt.f32.f16 flo, lo;\n\t"
+      "cvt.f32.f16 fhi, hi;\n\t"
+      "add.rn.f32 %0, flo, fhi;\n\t}"
+      : "=f"(out)
+      : "r"(e2m1x8_sum_h2(w0)), "r"(e2m1x8_sum_h2(w1)), "r"(e2m1x8_sum_h2(w2)), "r"(e2m1x8_sum_h2(w3)));
+  return out;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Shared-scale exponent: the smallest e with amax <= q * 2^e for q = mq * 2^eq (mq in [1,2)),
+// i.e. e = E(amax) - eq + [mant(amax) > mant(q)]; the OCP floor rule passes mant_q = 0xFFFFFFFF.
+// Exact integer arithmetic on the fp32 bit pattern; clamped to [-127, 127]; amax = 0 -> -127.
+// ------------------------------------------------------------------------------------------------
+struct ScaleRule {
+  int eq;          // binary exponent of the boundary q
+  uint32_t mq;     // its 23 mantissa bits (0xFFFFFFFF: never step up -> floor rule)
+};
+
+__device__ __forceinline__ int shared_exponent(float amax, ScaleRule r) {
+  uint32_t b = __float_as_uint(amax) & 0x7FFFFFFFu;
+  if (b == 0) return -127;
+  int E;
+  uint32_t m;
+  if (b >= 0x00800000u) {
+    E = (int)(b >> 23) - 127;
+    m = b & 0x007FFFFFu;
+  } else {  // subnormal: value = b * 2^-149
+    const int p = 31 - __clz(b);
+    E = p - 149;
+    m = (b << (23 - p)) & 0x007FFFFFu;
+  }
+  int e = E - r.eq + (m > r.mq ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^-e as an fp32 for e in [-127, 126] (a normal number).
+__device__ __forceinline__ float pow2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
+
+}  // namespace mxattn

@@ -1,0 +1,250 @@
+// quant.cu -- MXFP4 quantizers (rotation + quantization of Q/K, V along keys, and a plain
+// generic quantizer).  Memory-bound: every byte is read once and written once, loads and
+// stores are 16-byte vectors, FWHT butterflies run in registers and warp shuffles.
+//
+// Method: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for
+// MXFP4 Attention" -- Pith review page (axioms ledger: 32-element E2M1 groups with one E8M0
+// scale, round to nearest with saturation; Fig. 3: OCP floor [4,8), TFS (3,6], UOS
+// (3.625,7.25]; Fig. 1: fixed Hadamard rotation on Q/K) and the 10100.com article.
+//
+// Every product here is x * 2^-e (exact) and every sum is an fp32 butterfly with explicit
+// round-to-nearest intrinsics, so the codes are a deterministic function of the inputs.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mxattn {
+
+template <int DT>
+__device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid, float (&v)[8]) {
+  if (!valid) {
+#pragma unroll
+    for (int i = 0; i < 8; i++) v[i] = 0.f;
+    return;
+  }
+  if (DT == kBF16) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 a = p[0], b = p[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Q/K: Hadamard rotation + quantization along d into the packed QK operand layout.
+// D/8 threads per token row, 8 consecutive elements per thread; groups of 32 = 4 threads.
+// Grid: x over (B*H*T128*128) padded token rows, y = 0 for Q, 1 for K.
+// ------------------------------------------------------------------------------------------------
+template <int D, int DT>
+__global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
+  constexpr int TPR = D / 8;                 // threads per row
+  constexpr int ROWS = 256 / TPR;            // rows per block
+  const int t = threadIdx.x;
+  const int tl = t % TPR;                    // thread within the row
+  const int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;   // padded row id
+  const int64_t T128 = (a.N + 127) / 128;
+  const int64_t total = (int64_t)a.BH * T128 * 128;
+  const bool row_ok = prow < total;          // whole warps share this (ROWS multiple of 2)
+  const int64_t bh = prow / (T128 * 128);
+  const int tok = (int)(prow % (T128 * 128));
+  const bool valid = row_ok && tok < a.N;
+
+  const void* src = blockIdx.y == 0 ? a.q : a.k;
+  uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
+  uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
+
+  float v[8];
+  load8<DT>(src, ((int64_t)bh * a.N + (valid ? tok : 0)) * D + tl * 8, valid, v);
+
+  if (a.rotate) {
+    // stages h = 1, 2, 4 inside the thread
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        if ((i & h) == 0) {
+          const float x = v[i], y = v[i + h];
+          v[i] = __fadd_rn(x, y);
+          v[i + h] = __fsub_rn(x, y);
+        }
+      }
+    }
+    // stages h = 8 .. D/2 across the TPR lanes of the row (lane bit = h / 8)
+#pragma unroll
+    for (int hb = 1; hb < TPR; hb <<= 1) {
+      const bool upper = (tl & hb) != 0;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const float other = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
+        v[i] = upper ? __fsub_rn(other, v[i]) : __fadd_rn(v[i], other);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i++) v[i] = __fmul_rn(v[i], a.hadamard_scale);
+  }
+
+  // group amax over the 4 threads of a 32-element group
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; i++) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  const int e = shared_exponent(amax, a.rule);
+  const float inv = pow2_neg(e);
+  const uint32_t w = cvt_e2m1x8(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
+                                __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
+                                __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  if (!row_ok) return;
+  const int r = tok % 128;
+  const int64_t tile = bh * T128 + tok / 128;
+  const int c = tl / 4;                                   // group / 16-byte chunk
+  const int s = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
+  uint8_t* rowp = codes + (tile * 128 + r) * (D / 2);
+  *reinterpret_cast<uint32_t*>(rowp + ((c ^ s) * 16) + (tl % 4) * 4) = w;
+  if ((tl & 3) == 0) {
+    uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
+    atom[c] = (uint8_t)(e + 127);
+    if (D == 64) atom[c + 2] = 0;                         // unused scale slots
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// V: quantization along keys (32 consecutive tokens per channel) into the packed V operand
+// layout.  One block per (head, 64-key tile): the tile is staged through shared memory as
+// fp32 [64][D+1], then thread (channel c, half h) quantizes keys 32h..32h+31 of channel c.
+// ------------------------------------------------------------------------------------------------
+template <int D, int DT>
+__global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
+  __shared__ float tile[64][D + 1];
+  const int T64 = (a.N + 63) / 64;
+  const int T128 = (a.N + 127) / 128;
+  const int bh = blockIdx.x / T64;
+  const int j = blockIdx.x % T64;
+  const int t = threadIdx.x;
+  // stage: 64 tokens x D values, 8 values per thread-iteration
+  constexpr int VEC_PER_ROW = D / 8;
+  for (int idx = t; idx < 64 * VEC_PER_ROW; idx += 256) {
+    const int row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
+    const int tok = j * 64 + row;
+    float v[8];
+    load8<DT>(a.v, ((int64_t)bh * a.N + (tok < a.N ? tok : 0)) * D + cv * 8, tok < a.N, v);
+#pragma unroll
+    for (int i = 0; i < 8; i++) tile[row][cv * 8 + i] = v[i];
+  }
+  __syncthreads();
+  for (int item = t; item < 2 * D; item += 256) {
+    const int c = item % D, h = item / D;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(tile[h * 32 + i][c]));
+    const int e = shared_exponent(amax, a.rule);
+    const float inv = pow2_neg(e);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      const int b = h * 32 + q * 8;
+      w[q] = cvt_e2m1x8(__fmul_rn(tile[b + 0][c], inv), __fmul_rn(tile[b + 1][c], inv),
+                        __fmul_rn(tile[b + 2][c], inv), __fmul_rn(tile[b + 3][c], inv),
+                        __fmul_rn(tile[b + 4][c], inv), __fmul_rn(tile[b + 5][c], inv),
+                        __fmul_rn(tile[b + 6][c], inv), __fmul_rn(tile[b + 7][c], inv));
+    }
+    uint8_t* dst = a.v_codes + (((int64_t)bh * T64 + j) * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    uint8_t* atom = a.v_scales + ((int64_t)bh * T128 + j / 2) * 512;
+    atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
+    if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
+    // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
+    if (j == T64 - 1 && (j % 2) == 0) {
+      atom[(c % 32) * 16 + (c / 32) * 4 + 2 + h] = 0;
+      if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 + h] = 0;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Generic quantizer, plain layout: one thread per group of 32.
+// axis 0: groups along columns of a row; axis 1: groups along rows of a column (transposed out).
+// ------------------------------------------------------------------------------------------------
+template <int DT>
+__global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
+  const int64_t outer = a.axis == 0 ? a.rows : a.cols;
+  const int64_t inner = a.axis == 0 ? a.cols : a.rows;
+  const int64_t ng = (inner + 31) / 32;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= outer * ng) return;
+  // axis 1: consecutive threads take consecutive columns (coalesced); axis 0: consecutive groups
+  const int64_t o = a.axis == 0 ? gid / ng : gid % outer;
+  const int64_t g = a.axis == 0 ? gid % ng : gid / outer;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; i++) {
+    const int64_t in = g * 32 + i;
+    float x = 0.f;
+    if (in < inner) {
+      const int64_t idx = a.axis == 0 ? o * a.cols + in : in * a.cols + o;
+      if (DT == kBF16)
+        x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.x)[idx]);
+      else
+        x = reinterpret_cast<const float*>(a.x)[idx];
+    }
+    v[i] = x;
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = shared_exponent(amax, a.rule);
+  const float inv = pow2_neg(e);
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; q++)
+    w[q] = cvt_e2m1x8(__fmul_rn(v[q * 8 + 0], inv), __fmul_rn(v[q * 8 + 1], inv), __fmul_rn(v[q * 8 + 2], inv),
+                      __fmul_rn(v[q * 8 + 3], inv), __fmul_rn(v[q * 8 + 4], inv), __fmul_rn(v[q * 8 + 5], inv),
+                      __fmul_rn(v[q * 8 + 6], inv), __fmul_rn(v[q * 8 + 7], inv));
+  *reinterpret_cast<uint4*>(a.codes + (o * ng + g) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  a.scales[o * ng + g] = (uint8_t)(e + 127);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Launchers
+// ------------------------------------------------------------------------------------------------
+cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
+  const int64_t rows = (int64_t)a.BH * ((a.N + 127) / 128) * 128;
+  const int rows_per_block = 256 / (D / 8);
+  dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
+  if (D == 128 && dtype == kBF16) rotate_quant_qk_kernel<128, kBF16><<<grid, 256, 0, s>>>(a);
+  else if (D == 128) rotate_quant_qk_kernel<128, kFP32><<<grid, 256, 0, s>>>(a);
+  else if (dtype == kBF16) rotate_quant_qk_kernel<64, kBF16><<<grid, 256, 0, s>>>(a);
+  else rotate_quant_qk_kernel<64, kFP32><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s) {
+  const unsigned blocks = (unsigned)((int64_t)a.BH * ((a.N + 63) / 64));
+  if (D == 128 && dtype == kBF16) quant_v_kernel<128, kBF16><<<blocks, 256, 0, s>>>(a);
+  else if (D == 128) quant_v_kernel<128, kFP32><<<blocks, 256, 0, s>>>(a);
+  else if (dtype == kBF16) quant_v_kernel<64, kBF16><<<blocks, 256, 0, s>>>(a);
+  else quant_v_kernel<64, kFP32><<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_plain(const PlainQuantArgs& a, int dtype, cudaStream_t s) {
+  const int64_t outer = a.axis == 0 ? a.rows : a.cols;
+  const int64_t inner = a.axis == 0 ? a.cols : a.rows;
+  const int64_t groups = outer * ((inner + 31) / 32);
+  const unsigned blocks = (unsigned)((groups + 255) / 256);
+  if (dtype == kBF16) quant_plain_kernel<kBF16><<<blocks, 256, 0, s>>>(a);
+  else quant_plain_kernel<kFP32><<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace mxattn

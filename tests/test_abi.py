@@ -1,0 +1,75 @@
+"""The C-ABI library loads without a GPU and exports every symbol the header declares."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mxfp4_bit_attention_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "mxattn.h")).read()
+    return sorted(set(re.findall(r"MXATTN_API\s+[\w\s\*]+?\b(mxattn_\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp4_bit_attention_b200 import build
+    build.build()
+    return binding.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_host_only_calls(lib):
+    o = binding.COpts()
+    lib.mxattn_opts_default(ctypes.byref(o))
+    assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 64)
+    assert abs(o.qmax - 7.25) < 1e-7 and abs(o.rescale_tau - 8.0) < 1e-7
+    assert lib.mxattn_qk_codes_bytes(1, 2, 200, 128) == 2 * 2 * 128 * 64
+    assert lib.mxattn_qk_scales_bytes(1, 2, 200, 128) == 2 * 2 * 512
+    assert lib.mxattn_v_codes_bytes(1, 2, 200, 128) == 2 * 4 * 128 * 32
+    assert lib.mxattn_v_scales_bytes(1, 2, 200, 64) == 2 * 2 * 512
+    assert lib.mxattn_workspace_bytes(1, 1, 256, 96, ctypes.byref(o)) == 0
+    assert lib.mxattn_workspace_bytes(1, 40, 75600, 128, ctypes.byref(o)) > 256
+    assert lib.mxattn_status_string(5) == b"MXATTN_ERR_TIMEOUT"
+
+
+def test_validation_rejects_before_enqueue(lib):
+    """Invalid arguments return a status without touching the (fake) pointers."""
+    o = binding.COpts()
+    lib.mxattn_opts_default(ctypes.byref(o))
+    fake = ctypes.c_void_p(0x1000)
+    P = ctypes.byref(o)
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 96, 0.1, P, fake, None) == 1       # d
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 0, 64, 0.1, P, fake, None) == 1         # N
+    assert lib.mxattn_forward(None, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1       # null
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, -1.0, P, fake, None) == 1      # scale
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3       # no workspace
+    o.key_tile = 128
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
+    o.key_tile = 64
+    o.scale_rule = 3
+    o.qmax = 9.0
+    assert lib.mxattn_quant_v(fake, 1, 1, 256, 64, P, fake, fake, None) == 1
+    o.scale_rule = 7
+    assert lib.mxattn_quant_v(fake, 1, 1, 256, 64, P, fake, fake, None) == 1
+    o.scale_rule = 0
+    assert lib.mxattn_quantize_mxfp4(fake, 10, 10, 2, P, fake, fake, None) == 1
+    assert lib.mxattn_fp4_mma_probe(1, 1, 96, None) == 1
+
+
+def test_package_import_does_not_need_the_library(monkeypatch):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "lib_path", lambda: "/nonexistent/libmxattn.so")
+    with pytest.raises(ImportError):
+        binding.load()
