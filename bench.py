@@ -188,13 +188,13 @@ def cpu_oracle_sample(w, target_seconds: float):
     t0 = time.perf_counter()
     _, kd, vd = oracle.prepare_head(q[:1], k, v)
     prep = time.perf_counter() - t0
-    # calibrate rows on a small probe, then run the bounded sample
-    rows = [0]
+    # calibrate on one row per oracle thread, then run the bounded sample
+    probe = np.arange(cores, dtype=np.int64) * max(1, w.N // cores)
     t1 = time.perf_counter()
-    qd, _, _ = oracle.prepare_head(q[rows], k[:32], v[:32])
+    qd, _, _ = oracle.prepare_head(q[probe], k[:32], v[:32])
     oracle.attention_rows(qd, kd, vd, s, w.key_tile, tau=8.0)
-    per_row = max(time.perf_counter() - t1, 1e-4)
-    nrows = int(max(1, min(w.N, (target_seconds - prep) / per_row)))
+    per_row = max(time.perf_counter() - t1, 1e-4) / len(probe)
+    nrows = int(max(cores, min(w.N, (target_seconds - prep) / per_row)))
     sel = np.linspace(0, w.N - 1, nrows).astype(np.int64)
     t2 = time.perf_counter()
     qd, _, _ = oracle.prepare_head(q[sel], k[:32], v[:32])

@@ -182,6 +182,27 @@ MXATTN_API mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const ui
                                      void* out, void* stream);
 
 /*
+ * Diagnostic variant of mxattn_attention_mxfp4: identical results, and the CTA
+ * that owns query tile dump_qt (128 rows) of head dump_bh (index into B*H)
+ * also writes its internal state to `dump` (device buffer of
+ * mxattn_attention_dump_bytes(N, d) bytes, 16-byte aligned), in this order:
+ *   S of key tiles 0 and 1       fp32 [2][128][64], raw Q^ K^T from the MMA
+ *   P^ codes of every key tile   [ceil(N/64)][128][32] bytes, keys in order,
+ *                                element 2i in the low nibble
+ *   P^ scales of every key tile  [ceil(N/64)][128][2] E8M0 bytes (groups 0, 1)
+ *   O~ accumulator               fp32 [128][d] before the division by l
+ *   l, m                         fp32 [128] each; m = running max of
+ *                                S * softmax_scale * log2(e) used for P~
+ * (the O~, l, m block starts at the next 16-byte boundary).  Used to measure
+ * how many P^ codes differ from the oracle's; the paper has no counterpart.
+ */
+MXATTN_API size_t mxattn_attention_dump_bytes(int N, int d);
+MXATTN_API mxattn_status mxattn_attention_mxfp4_dump(
+    const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes, const uint8_t* k_scales,
+    const uint8_t* v_codes, const uint8_t* v_scales, int B, int H, int N, int d, float softmax_scale,
+    const mxattn_opts* opts, void* out, int dump_bh, int dump_qt, uint8_t* dump, void* stream);
+
+/*
  * The whole forward pass: mxattn_hadamard_quant_qk + mxattn_quant_v into
  * the workspace, then mxattn_attention_mxfp4.  d in {64, 128}, N >= 1.
  */

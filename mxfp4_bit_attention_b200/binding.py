@@ -24,7 +24,8 @@ EXPORTS = (
     "mxattn_qk_scales_bytes", "mxattn_v_codes_bytes", "mxattn_v_scales_bytes",
     "mxattn_workspace_init", "mxattn_quantize_mxfp4", "mxattn_hadamard_quant_qk",
     "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
-    "mxattn_status_string", "mxattn_fp4_mma_probe",
+    "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
+    "mxattn_attention_mxfp4_dump",
 )
 
 
@@ -85,6 +86,8 @@ def load():
         "mxattn_get_device_error": ([PO, P], i32),
         "mxattn_status_string": ([i32], ctypes.c_char_p),
         "mxattn_fp4_mma_probe": ([i32, i32, i32, P], i32),
+        "mxattn_attention_dump_bytes": ([i32, i32], sz),
+        "mxattn_attention_mxfp4_dump": ([P, P, P, P, P, P, i32, i32, i32, i32, f32, PO, P, i32, i32, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -200,6 +203,47 @@ def mxattn_attention_mxfp4(ops, B, H, N, d, softmax_scale, out, opts: Opts | Non
         _ptr(ops["v_codes"]), _ptr(ops["v_scales"]), B, H, N, d, float(softmax_scale), ctypes.byref(c),
         _ptr(out), _stream(stream)))
     return out
+
+
+def dump_layout(N: int, d: int) -> dict:
+    """Byte offsets of the diagnostic dump (mirrors the header's description)."""
+    T64 = (N + 63) // 64
+    p_codes = 2 * 128 * 64 * 4
+    p_scales = p_codes + T64 * 128 * 32
+    o = (p_scales + T64 * 128 * 2 + 15) // 16 * 16
+    l = o + 128 * d * 4
+    m = l + 128 * 4
+    return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "total": m + 128 * 4}
+
+
+def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, dump_qt=0, opts=None,
+                                workspace=None, stream=None):
+    """mxattn_attention_mxfp4 plus the diagnostic dump of one CTA; returns the dump as a dict
+    of numpy arrays (S tiles, P codes unpacked one per byte, P scales, O accumulator, l, m)."""
+    import numpy as np
+    import torch
+    ws = workspace if workspace is not None else torch.zeros(256, dtype=torch.uint8, device=out.device)
+    nbytes = int(load().mxattn_attention_dump_bytes(N, d))
+    dump = torch.zeros(nbytes, dtype=torch.uint8, device=out.device)
+    c = _copts(opts, _dtype_code(out), ws)
+    _check("mxattn_attention_mxfp4_dump", load().mxattn_attention_mxfp4_dump(
+        _ptr(ops["q_codes"]), _ptr(ops["q_scales"]), _ptr(ops["k_codes"]), _ptr(ops["k_scales"]),
+        _ptr(ops["v_codes"]), _ptr(ops["v_scales"]), B, H, N, d, float(softmax_scale), ctypes.byref(c),
+        _ptr(out), dump_bh, dump_qt, _ptr(dump), _stream(stream)))
+    torch.cuda.synchronize()
+    raw = dump.cpu().numpy()
+    L = dump_layout(N, d)
+    T64 = (N + 63) // 64
+    pc = raw[L["p_codes"]:L["p_scales"]].reshape(T64, 128, 32)
+    codes = np.empty((T64, 128, 64), np.uint8)
+    codes[..., 0::2] = pc & 0x0F
+    codes[..., 1::2] = pc >> 4
+    return {"s": raw[:L["p_codes"]].view(np.float32).reshape(2, 128, 64),
+            "p_codes": codes,
+            "p_scales": raw[L["p_scales"]:L["p_scales"] + T64 * 256].reshape(T64, 128, 2),
+            "o": raw[L["o"]:L["l"]].view(np.float32).reshape(128, d),
+            "l": raw[L["l"]:L["m"]].view(np.float32).copy(),
+            "m": raw[L["m"]:L["total"]].view(np.float32).copy()}
 
 
 def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None, stream=None):

@@ -227,6 +227,47 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
   a.wait_budget = kWaitBudgetCycles;
+  a.dump = nullptr;
+  a.dump_bh = a.dump_qt = -1;
+  return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
+}
+
+size_t mxattn_attention_dump_bytes(int N, int d) {
+  if (!sizes_ok(1, 1, N, d)) return 0;
+  return DumpLayout(d, (int)t64(N)).total;
+}
+
+mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                          const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales,
+                                          int B, int H, int N, int d, float softmax_scale, const mxattn_opts* o,
+                                          void* out, int dump_bh, int dump_qt, uint8_t* dump, void* stream) {
+  if (dump == nullptr || !aligned16(dump) || dump_bh < 0 || dump_qt < 0) return MXATTN_ERR_INVALID_ARG;
+  if (!sizes_ok(B, H, N, d) || dump_bh >= B * H || dump_qt >= t128(N)) return MXATTN_ERR_INVALID_ARG;
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !v_codes || !v_scales || !out) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  st = check_workspace(o, kStatusBytes);
+  if (st != MXATTN_OK) return st;
+  AttnArgs a;
+  a.q_codes = q_codes;
+  a.q_scales = q_scales;
+  a.k_codes = k_codes;
+  a.k_scales = k_scales;
+  a.v_codes = v_codes;
+  a.v_scales = v_scales;
+  a.out = out;
+  a.status = reinterpret_cast<int*>(o->workspace);
+  a.BH = B * H;
+  a.N = N;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+  a.tau = o->rescale_tau;
+  a.pnq = o->pnq;
+  make_rule(o, &a.rule);
+  a.wait_budget = kWaitBudgetCycles;
+  a.dump = dump;
+  a.dump_bh = dump_bh;
+  a.dump_qt = dump_qt;
   return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
 }
 

@@ -215,7 +215,10 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     const int row = threadIdx.x;  // TMEM lane and query row within the tile
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const float c = a.scale_log2;
-    float m2 = -INFINITY;  // running max of S*c (log2 units) actually used for the exponent
+    const bool dumping = a.dump != nullptr && bh == a.dump_bh && qt == a.dump_qt;
+    const DumpLayout dl(D, T64);
+    float sm = -INFINITY;  // running max of S used for the exponent (raw MMA units)
+    float m2 = -INFINITY;  // the same in log2 units, fl32(sm * c)
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < T64; j++) {
@@ -229,6 +232,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_S_FREE));
+      if (dumping && j < 2) {
+        float* ds = reinterpret_cast<float*>(a.dump + dl.s) + ((size_t)j * 128 + row) * 64;
+        for (int i = 0; i < 32; i++) {
+          ds[i] = __uint_as_float(s0[i]);
+          ds[32 + i] = __uint_as_float(s1[i]);
+        }
+      }
 
       const int valid = min(kBN, a.N - j * kBN);
       float gmax[2];
@@ -242,18 +252,23 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
         gmax[g] = mx;
       }
-      const float mt = fmaxf(gmax[0], gmax[1]) * c;
+      // Running max kept in raw S units (sm) and in log2 units (m2 = fl32(sm * c)).  A group's
+      // maximum is taken as 2^((gmax - sm) * c): exactly 1 for the group that holds the running
+      // max, as exp(0) is in the oracle, so scale rules whose boundaries sit on powers of two
+      // (OCP, q = 4 or 8) decide it the same way.
+      const float mt_raw = fmaxf(gmax[0], gmax[1]);
       const bool first = (j == 0);
-      const bool move = first || (mt > m2 + a.tau);
-      const float mnew = move ? mt : m2;
-      const float alpha = first ? 0.f : (move ? ex2_approx(m2 - mnew) : 1.f);
-      m2 = mnew;
+      const bool move = first || (mt_raw * c > m2 + a.tau);
+      const float sm_new = move ? mt_raw : sm;
+      const float alpha = first ? 0.f : (move ? ex2_approx((sm - sm_new) * c) : 1.f);
+      sm = sm_new;
+      m2 = sm * c;
 
       int e[2];
       float bias[2];
 #pragma unroll
       for (int g = 0; g < 2; g++) {
-        const float amax = gmax[g] == -INFINITY ? 0.f : ex2_approx(fmaf(gmax[g], c, -m2));
+        const float amax = gmax[g] == -INFINITY ? 0.f : ex2_approx((gmax[g] - sm) * c);
         e[g] = shared_exponent(amax, a.rule);
         bias[g] = m2 + (float)e[g];
       }
@@ -275,9 +290,15 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       float lsum = 0.f;
 #pragma unroll
       for (int g = 0; g < 2; g++) {
-        const float sc = e[g] > -127 ? __uint_as_float((uint32_t)(e[g] + 127) << 23) : 0.f;
-        const float gs = PNQ ? e2m1x32_sum(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]) : psum[g];
-        lsum += gs * sc;
+        if (PNQ) {
+          // sum of the quantized tile: (integer half-units) * 2^(e - 1), both factors exact
+          const uint32_t halves = e2m1x32_sum_halves(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+          const float sc = e[g] > -126 ? __uint_as_float((uint32_t)(e[g] + 126) << 23) : 0.f;
+          lsum += (float)halves * sc;
+        } else {
+          const float sc = e[g] > -127 ? __uint_as_float((uint32_t)(e[g] + 127) << 23) : 0.f;
+          lsum += psum[g] * sc;
+        }
       }
       l = alpha * l + lsum;
 
@@ -309,6 +330,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_P_FULL));
+      if (dumping) {
+        uint32_t* dp = reinterpret_cast<uint32_t*>(a.dump + dl.p_codes + ((size_t)j * 128 + row) * 32);
+        for (int i = 0; i < 8; i++) dp[i] = w[i];
+        uint8_t* dsf = a.dump + dl.p_scales + ((size_t)j * 128 + row) * 2;
+        dsf[0] = (uint8_t)(e[0] + 127);
+        dsf[1] = (uint8_t)(e[1] + 127);
+      }
     }
     if (ok) {
       ok = mbar_wait(bar(L::B_O_DONE), (T64 - 1) & 1, abort_flag, a.wait_budget);
@@ -325,6 +353,14 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         uint32_t o[32];
         tmem_ld32(tl + L::T_O + 32 * cc, o);
         tmem_wait_ld();
+        if (dumping) {
+          float* d_o = reinterpret_cast<float*>(a.dump + dl.o) + (size_t)row * D + 32 * cc;
+          for (int i = 0; i < 32; i++) d_o[i] = __uint_as_float(o[i]);
+          if (cc == 0) {
+            reinterpret_cast<float*>(a.dump + dl.l)[row] = l;
+            reinterpret_cast<float*>(a.dump + dl.m)[row] = m2;
+          }
+        }
         if (store) {
           if (DT == kBF16) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + obase + 32 * cc);

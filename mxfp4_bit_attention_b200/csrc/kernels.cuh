@@ -55,6 +55,27 @@ struct AttnArgs {
   int pnq;
   ScaleRule rule;
   long long wait_budget; // SM clock cycles a bounded wait may spin before giving up
+  uint8_t* dump;         // optional diagnostic dump of one CTA (layout: see dump_layout below)
+  int dump_bh, dump_qt;
+};
+
+// Diagnostic dump of the CTA (dump_bh, dump_qt), byte offsets for head dim D and T64 key tiles:
+//   [0, 64K)               S of key tiles 0 and 1, fp32 [2][128][64] (as read from TMEM)
+//   P codes                [T64][128][32] bytes, logical key order (element 2i in the low nibble)
+//   P scales               [T64][128][2] bytes (E8M0 of key groups 0 and 1 of the tile)
+//   O accumulator          [128][D] fp32, before the division by l
+//   l, m                   [128] fp32 each (m in log2 units: running max of S * scale * log2 e)
+struct DumpLayout {
+  size_t s, p_codes, p_scales, o, l, m, total;
+  __host__ __device__ DumpLayout(int D, int T64) {
+    s = 0;
+    p_codes = 2 * 128 * 64 * 4;
+    p_scales = p_codes + (size_t)T64 * 128 * 32;
+    o = (p_scales + (size_t)T64 * 128 * 2 + 15) / 16 * 16;
+    l = o + (size_t)128 * D * 4;
+    m = l + 128 * 4;
+    total = m + 128 * 4;
+  }
 };
 
 // Status words written by a kernel whose bounded wait expired.

@@ -203,39 +203,21 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
   return out;
 }
 
-// Sum of the eight E2M1 values packed in a 32-bit word, as an f16x2 pair of partial sums.
-// Exact: every partial sum is a multiple of 0.5 below 64.
-__device__ __forceinline__ uint32_t e2m1x8_sum_h2(uint32_t w) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
-      "add.rn.f16x2 h0, h0, h1;\n\t"
-      "add.rn.f16x2 h2, h2, h3;\n\t"
-      "add.rn.f16x2 %0, h0, h2;\n\t}"
-      : "=r"(out)
-      : "r"(w));
-  return out;
-}
-
-// Sum of the 32 E2M1 values packed in four words, as fp32 (exact: at most 32 * 6 = 192, a
-// multiple of 0.5, so every f16 partial sum is exact).
-__device__ __forceinline__ float e2m1x32_sum(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
-  float out;
-  asm("{\n\t.reg .b32 a, b, c, d;\n\t.reg .b16 lo, hi;\n\t.reg .f32 flo, fhi;\n\t"
-      "add.rn.f16x2 a, %1, %2;\n\t"
-      "add.rn.f16x2 b, %3, %4;\n\t"
-      "add.rn.f16x2 c, a, b;\n\t"
-      "mov.b32 {lo, hi}, c;\n\t"
-      "cvt.f32.f16 flo, lo;\n\t"
-      "cvt.f32.f16 fhi, hi;\n\t"
-      "add.rn.f32 %0, flo, fhi;\n\t}"
-      : "=f"(out)
-      : "r"(e2m1x8_sum_h2(w0)), "r"(e2m1x8_sum_h2(w1)), "r"(e2m1x8_sum_h2(w2)), "r"(e2m1x8_sum_h2(w3)));
-  return out;
+// Sum of 32 non-negative E2M1 codes (four packed words), in units of 0.5, exact.
+// Each nibble (magnitude index 0..7, sign bit clear) selects its value in half-units
+// {0, 1, 2, 3, 4, 6, 8, 12} from an 8-byte table with one byte permute per 4 codes, and
+// dp4a adds the four bytes into an integer accumulator.
+__device__ __forceinline__ uint32_t e2m1x32_sum_halves(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  constexpr uint32_t kLo = 0x03020100u;  // half-units of codes 0..3
+  constexpr uint32_t kHi = 0x0C080604u;  // half-units of codes 4..7
+  const uint32_t w[4] = {w0, w1, w2, w3};
+  uint32_t acc = 0;
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    acc = __dp4a(__byte_perm(kLo, kHi, w[i]), 0x01010101u, acc);
+    acc = __dp4a(__byte_perm(kLo, kHi, w[i] >> 16), 0x01010101u, acc);
+  }
+  return acc;
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
