@@ -211,6 +211,31 @@ MXATTN_API mxattn_status mxattn_forward(const void* q, const void* k, const void
                              void* stream);
 
 /*
+ * mxattn_forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory: a process whose memory manager has already reserved
+ * the GPU's memory (a cudaMalloc would fail or fragment its pool), or a plain C
+ * caller without allocator plumbing.  The paper has no counterpart; this is a
+ * deployment variant of the same pass.
+ *  - Scratch (packed Q/K/V operands and the status block) comes from a fixed
+ *    64 MiB array inside the library; every GPU that loads the library holds it
+ *    until the process exits.  Problems whose mxattn_workspace_bytes() exceeds
+ *    64 MiB (at d = 128, about 300k query rows summed over B*H) are rejected
+ *    with MXATTN_ERR_WORKSPACE before anything is enqueued.
+ *  - opts->workspace and opts->workspace_bytes are ignored.  No memory is
+ *    allocated or freed by this call.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - All calls share the one array: calls that may overlap on the GPU (other
+ *    streams, other host threads) race and corrupt each other's results;
+ *    serialize them.  The status block is cleared at the start of every call,
+ *    so a bounded-wait expiry is not reported through mxattn_get_device_error.
+ *  - q, k, v, out: as mxattn_forward, on the current device.
+ */
+MXATTN_API mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v, int B, int H,
+                                                int N, int d, float softmax_scale, const mxattn_opts* opts,
+                                                void* out, void* stream);
+
+/*
  * Synchronize `stream`, read the workspace status block and clear it.
  * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
  * last call (its output is then undefined), MXATTN_OK otherwise.

@@ -25,7 +25,7 @@ EXPORTS = (
     "mxattn_workspace_init", "mxattn_quantize_mxfp4", "mxattn_hadamard_quant_qk",
     "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
-    "mxattn_attention_mxfp4_dump",
+    "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc",
 )
 
 
@@ -88,6 +88,7 @@ def load():
         "mxattn_fp4_mma_probe": ([i32, i32, i32, P], i32),
         "mxattn_attention_dump_bytes": ([i32, i32], sz),
         "mxattn_attention_mxfp4_dump": ([P, P, P, P, P, P, i32, i32, i32, i32, f32, PO, P, i32, i32, P, P], i32),
+        "mxattn_forward_noalloc": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -256,6 +257,22 @@ def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=No
     ws = workspace if workspace is not None else new_workspace(B, H, N, d, opts, q.device)
     c = _copts(opts, _dtype_code(q), ws)
     _check("mxattn_forward", load().mxattn_forward(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def mxattn_forward_noalloc(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, stream=None):
+    """mxattn_forward with the library's fixed internal scratch instead of a workspace: for
+    callers that cannot allocate device memory.  Problems needing more than the fixed scratch
+    raise MXAttnError(MXATTN_ERR_WORKSPACE); concurrent calls on one device race."""
+    import torch
+    B, H, N, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    out = out if out is not None else torch.empty_like(q)
+    c = _copts(opts, _dtype_code(q))
+    _check("mxattn_forward_noalloc", load().mxattn_forward_noalloc(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
         _stream(stream)))
     return out

@@ -1,0 +1,61 @@
+// noalloc.cu -- mxattn_forward_noalloc: the whole forward pass with its scratch memory (packed
+// Q/K/V operands and the status block) taken from a fixed array compiled into the library
+// instead of a caller-provided workspace.
+//
+// Some callers cannot hand the library a device buffer: code that runs under an external memory
+// manager which has already reserved the GPU's memory (a serving process that pre-allocates its
+// whole HBM budget, where a cudaMalloc would fail or fragment that pool), or a plain C caller with
+// no allocator plumbing at all.  This entry point allocates nothing: the scratch is a
+// file-scope __device__ array of kNoAllocScratchBytes, which every GPU that loads the library
+// holds until the process exits.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/mxattn.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 64u << 20;  // 64 MiB per device
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device.  In host code the symbol name
+// is only a host-side stand-in, so the address must come from cudaGetSymbolAddress with the
+// device current.
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+mxattn_status scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MXATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MXATTN_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MXATTN_OK;
+}
+
+}  // namespace
+
+extern "C" MXATTN_API mxattn_status mxattn_forward_noalloc(const void* q, const void* k, const void* v, int B,
+                                                           int H, int N, int d, float softmax_scale,
+                                                           const mxattn_opts* opts, void* out, void* stream) {
+  if (opts == nullptr) return MXATTN_ERR_INVALID_ARG;
+  const size_t need = mxattn_workspace_bytes(B, H, N, d, opts);
+  if (need == 0) return MXATTN_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return MXATTN_ERR_WORKSPACE;  // problem larger than the fixed scratch
+  void* scratch = nullptr;
+  const mxattn_status st = scratch_for_current_device(&scratch);
+  if (st != MXATTN_OK) return st;
+  mxattn_opts o = *opts;
+  o.workspace = scratch;
+  o.workspace_bytes = kNoAllocScratchBytes;
+  // The status block must start at zero; the packed operands are fully rewritten by the quantizers.
+  if (mxattn_workspace_init(&o, stream) != MXATTN_OK) return MXATTN_ERR_CUDA;
+  return mxattn_forward(q, k, v, B, H, N, d, softmax_scale, &o, out, stream);
+}
