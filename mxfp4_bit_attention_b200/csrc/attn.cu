@@ -14,9 +14,14 @@
 //   warps 0-3          one query row per thread: read S from TMEM, online max (optionally lazy,
 //                      threshold tau in log2 units), P~ = 2^(S*c - m) folded with the MXFP4 scale
 //                      of each 32-key group, E2M1 codes of P~ written to shared memory in the
-//                      MMA operand layout, group scales written as a scale atom, l updated from
-//                      the quantized codes (PNQ) or from P~ (direct placement), O~ rescaled in
+//                      MMA operand layout, group scales written as a scale atom, O~ rescaled in
 //                      TMEM when the running max moves, and finally O = O~ / l.
+// PNQ row sum: V^'s operand image carries 16 extra rows after its d channel rows, the first
+// all ones (scale 2^0), so the PV MMA also accumulates l = sum_k P^_k into O~ column d, with the
+// same codes, the same scales and the same rescaling as the output: the row sum is the sum of
+// the quantized tile by construction.  Direct placement (pnq = 0) sums P~ in registers instead.
+// The exp2s are split between MUFU (ex2.approx) and an FMA-pipe polynomial so that neither
+// pipe alone bounds the softmax.
 // Two CTAs share an SM (256 TMEM columns each), so one CTA's softmax overlaps the other's MMAs.
 // Every wait is bounded; on expiry the CTA records a status word, drains its in-flight copies
 // and MMAs, frees its TMEM and exits.
@@ -28,11 +33,19 @@
 
 namespace mxattn {
 
-constexpr int kBM = 128;      // query rows per CTA
-constexpr int kBN = 64;       // keys per tile
-constexpr int kStages = 4;    // K/V ring depth
-constexpr int kThreads = 192; // 4 softmax warps, producer warp, MMA warp
+constexpr int kBM = 128;        // query rows per CTA
+constexpr int kBN = 64;         // keys per tile
+constexpr int kStages = 4;      // K/V shared-memory ring depth
+constexpr int kSfSlots = 3;     // K/V scale-factor slots in TMEM (reuse distance 3 tiles)
+constexpr int kThreads = 192;   // 4 softmax warps, producer warp, MMA warp
+constexpr int kOnesRows = 16;   // rows appended to V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 256;
+#ifndef MXATTN_POLY_WORDS
+#define MXATTN_POLY_WORDS 0
+#endif
+// Of the four 8-key words of each 32-key group, this many take their exp2 from the FMA-pipe
+// polynomial instead of MUFU.
+constexpr int kPolyWords = MXATTN_POLY_WORDS;
 
 template <int D>
 struct Layout {
@@ -40,14 +53,16 @@ struct Layout {
   static constexpr int Q_BYTES = kBM * D / 2;
   static constexpr int K_BYTES = kBN * D / 2;
   static constexpr int V_BYTES = D * kBN / 2;
-  static constexpr int STAGE_BYTES = K_BYTES + V_BYTES;
+  static constexpr int ONES_BYTES = kOnesRows * kBN / 2;
+  static constexpr int STAGE_BYTES = K_BYTES + V_BYTES + ONES_BYTES;
   static constexpr int Q_CODES = 0;
   static constexpr int STAGE0 = Q_BYTES;
   static constexpr int P_CODES = STAGE0 + kStages * STAGE_BYTES;
   static constexpr int P_BYTES = kBM * kBN / 2;
   static constexpr int SF_Q = P_CODES + P_BYTES;
   static constexpr int SF_P = SF_Q + 512;
-  static constexpr int SF_K = SF_P + 512;
+  static constexpr int SF_ONES = SF_P + 512;   // scale atom of the ones rows (constant)
+  static constexpr int SF_K = SF_ONES + 512;
   static constexpr int SF_V = SF_K + kStages * 512;
   static constexpr int BARS = SF_V + kStages * 512;
   enum {
@@ -67,14 +82,15 @@ struct Layout {
   // slack for aligning the base; at least 80 KB so that no third CTA (which would block in
   // tcgen05.alloc until a neighbour frees its columns) becomes resident on an SM
   static constexpr int DYN_SMEM = TOTAL + 1024 > 80 * 1024 ? TOTAL + 1024 : 80 * 1024;
+  static_assert(STAGE_BYTES % 512 == 0, "K tiles need 512-byte alignment");
   // tensor memory columns
   static constexpr uint32_t T_S = 0;
-  static constexpr uint32_t T_O = 64;
-  static constexpr uint32_t T_SFQ = 64 + D;
+  static constexpr uint32_t T_O = 64;                      // O~: D columns, then l at column D
+  static constexpr uint32_t T_SFQ = T_O + D + kOnesRows;
   static constexpr uint32_t T_SFP = T_SFQ + 4;
-  static constexpr uint32_t T_SFK = T_SFP + 4;
-  static constexpr uint32_t T_SFV = T_SFK + 4 * kStages;
-  static_assert(T_SFV + 4 * kStages <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t T_SFK = T_SFP + 4;             // kSfSlots x 4 columns
+  static constexpr uint32_t T_SFV = T_SFK + 4 * kSfSlots;  // kSfSlots x 8 columns (V atom + ones atom)
+  static_assert(T_SFV + 8 * kSfSlots <= kTmemCols, "TMEM budget");
   static constexpr uint32_t QK_LAYOUT = D == 128 ? kLayoutSW64 : kLayoutSW32;
 };
 
@@ -83,9 +99,62 @@ __device__ __forceinline__ void raise_abort(volatile int* flag, int* status, int
   if (atomicCAS(status, 0, kStatusTimeout) == 0) atomicExch(status + 1, where);
 }
 
+// Group maximum of 32 raw S values (MASK: keys at index >= valid are excluded).
+template <bool MASK>
+__device__ __forceinline__ float group_max(const uint32_t (&s)[32], int base, int valid) {
+  float a = -INFINITY, b = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4) {
+    float v0 = __uint_as_float(s[i]), v1 = __uint_as_float(s[i + 1]);
+    float v2 = __uint_as_float(s[i + 2]), v3 = __uint_as_float(s[i + 3]);
+    if (MASK) {
+      v0 = base + i < valid ? v0 : -INFINITY;
+      v1 = base + i + 1 < valid ? v1 : -INFINITY;
+      v2 = base + i + 2 < valid ? v2 : -INFINITY;
+      v3 = base + i + 3 < valid ? v3 : -INFINITY;
+    }
+    a = fmax3(a, v0, v1);
+    b = fmax3(b, v2, v3);
+  }
+  return fmaxf(a, b);
+}
+
+// E2M1 codes of one group of 32: p = 2^(S*c - bias), 4 packed words.  Direct placement also
+// accumulates the unquantized p.
+template <bool MASK, bool SUM>
+__device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, int valid, float c, float bias,
+                                            uint32_t* w, float& psum) {
+  const float2 cc = make_float2(c, c);
+  const float2 nb = make_float2(-bias, -bias);
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float2 x =
+          __ffma2_rn(make_float2(__uint_as_float(s[q * 8 + i]), __uint_as_float(s[q * 8 + i + 1])), cc, nb);
+      if (q >= 4 - kPolyWords) {
+        const float2 y = exp2_poly2(x);
+        p[i] = y.x;
+        p[i + 1] = y.y;
+      } else {
+        p[i] = ex2_approx(x.x);
+        p[i + 1] = ex2_approx(x.y);
+      }
+      if (MASK) {
+        p[i] = base + q * 8 + i < valid ? p[i] : 0.f;
+        p[i + 1] = base + q * 8 + i + 1 < valid ? p[i + 1] : 0.f;
+      }
+      if (SUM) psum += p[i] + p[i + 1];
+    }
+    w[q] = cvt_e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+  }
+}
+
 template <int D, int DT, bool PNQ>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
   using L = Layout<D>;
+  constexpr int NV = PNQ ? D + kOnesRows : D;  // N of the PV MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -112,6 +181,18 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     mbar_init(bar(L::B_O_DONE), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     fence_mbar_init();
+  }
+  if (PNQ) {
+    // the ones rows of every stage (row 0: code 1.0 = 0x2 in every nibble; rows 1..15: zero) and
+    // their scale atom (row 0, every key group: 2^0; everything else zero)
+    for (int i = threadIdx.x; i < kStages * L::ONES_BYTES / 4; i += kThreads) {
+      const int st = i / (L::ONES_BYTES / 4), off = i % (L::ONES_BYTES / 4);
+      reinterpret_cast<uint32_t*>(smem + L::STAGE0 + st * L::STAGE_BYTES + L::K_BYTES + L::V_BYTES)[off] =
+          off < (kBN / 2) / 4 ? 0x22222222u : 0u;
+    }
+    for (int i = threadIdx.x; i < 512 / 4; i += kThreads)
+      reinterpret_cast<uint32_t*>(smem + L::SF_ONES)[i] = i == 0 ? 0x7F7F7F7Fu : 0u;
+    fence_proxy_async_smem();
   }
   if (warp == 5) {
     tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
@@ -164,16 +245,26 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       if (ok) {
         tc_fence_after();
         tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
+        if (PNQ)
+          for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
         const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
         const uint64_t pdesc = smem_desc(sb + L::P_CODES, 16, 8 * (kBN / 2), kLayoutSW32);
         for (int j = 0; j <= T64; j++) {
           if (j < T64) {
-            const int s = j % kStages;
+            const int s = j % kStages, f = j % kSfSlots;
             ok = mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget);
             if (!ok) break;
             tc_fence_after();
-            tmem_cp_sf_atom(tmem + L::T_SFK + 4 * s, sb + L::SF_K + 512 * s);
-            tmem_cp_sf_atom(tmem + L::T_SFV + 4 * s, sb + L::SF_V + 512 * s);
+            if (PNQ && D == 64) {
+              // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
+              // channels >= d are zero): give it scale 2^0 for all four key groups
+              *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * s + 8) = 0x7F7F7F7Fu;
+              fence_proxy_async_smem();
+            }
+            // slot f was last read by the MMAs of tile j-3, complete since the softmax saw
+            // O_DONE(j-3) before releasing P(j-2), which this thread waited for
+            tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
+            tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f, sb + L::SF_V + 512 * s);
             if (j > 0) {
               ok = mbar_wait(bar(L::B_S_FREE), (j - 1) & 1, abort_flag, a.wait_budget);
               if (!ok) break;
@@ -186,20 +277,20 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
               // scale bytes 2kb and 2kb+1 of each row's scale word.
               mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
                        mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
-                       tmem + L::T_SFK + 4 * s + 2 * (j & 1), kb > 0 ? 1u : 0u);
+                       tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
             }
             mma_commit(bar(L::B_S_FULL));
           }
           if (j > 0) {
-            const int jp = j - 1, sp = jp % kStages;
+            const int jp = j - 1, sp = jp % kStages, fp = jp % kSfSlots;
             ok = mbar_wait(bar(L::B_P_FULL), jp & 1, abort_flag, a.wait_budget);
             if (!ok) break;
             tc_fence_after();
             tmem_cp_sf_atom(tmem + L::T_SFP, sb + L::SF_P);
             const uint64_t vdesc =
                 smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
-            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, D, 0, 2 * (jp & 1)), tmem + L::T_SFP,
-                     tmem + L::T_SFV + 4 * sp, jp > 0 ? 1u : 0u);
+            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP,
+                     tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
             mma_commit(bar(L::B_O_DONE));
             mma_commit(bar(L::B_KV_EMPTY + sp));
           }
@@ -219,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     const DumpLayout dl(D, T64);
     float sm = -INFINITY;  // running max of S used for the exponent (raw MMA units)
     float m2 = -INFINITY;  // the same in log2 units, fl32(sm * c)
-    float l = 0.f;
+    float l = 0.f;         // direct placement only (PNQ keeps l in O~ column D)
     bool ok = true;
     for (int j = 0; j < T64; j++) {
       ok = mbar_wait(bar(L::B_S_FULL), j & 1, abort_flag, a.wait_budget);
@@ -241,16 +332,14 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
 
       const int valid = min(kBN, a.N - j * kBN);
+      const bool full = valid == kBN;  // uniform across the CTA
       float gmax[2];
-#pragma unroll
-      for (int g = 0; g < 2; g++) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-          const float s = __uint_as_float(g == 0 ? s0[i] : s1[i]);
-          mx = fmaxf(mx, (g * 32 + i < valid) ? s : -INFINITY);
-        }
-        gmax[g] = mx;
+      if (full) {
+        gmax[0] = group_max<false>(s0, 0, valid);
+        gmax[1] = group_max<false>(s1, 32, valid);
+      } else {
+        gmax[0] = group_max<true>(s0, 0, valid);
+        gmax[1] = group_max<true>(s1, 32, valid);
       }
       // Running max kept in raw S units (sm) and in log2 units (m2 = fl32(sm * c)).  A group's
       // maximum is taken as 2^((gmax - sm) * c): exactly 1 for the group that holds the running
@@ -274,33 +363,22 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
       uint32_t w[8];
       float psum[2] = {0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < 8; q++) {
-        const int g = q / 4;
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-          const int idx = q * 8 + i;
-          const float x = fmaf(__uint_as_float(g == 0 ? s0[idx] : s1[idx - 32]), c, -bias[g]);
-          p[i] = idx < valid ? ex2_approx(x) : 0.f;
-          if (!PNQ) psum[g] += p[i];
-        }
-        w[q] = cvt_e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+      if (full) {
+        group_codes<false, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
+        group_codes<false, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
+      } else {
+        group_codes<true, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
+        group_codes<true, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
       }
-      float lsum = 0.f;
+      if (!PNQ) {
+        float lsum = 0.f;
 #pragma unroll
-      for (int g = 0; g < 2; g++) {
-        if (PNQ) {
-          // sum of the quantized tile: (integer half-units) * 2^(e - 1), both factors exact
-          const uint32_t halves = e2m1x32_sum_halves(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-          const float sc = e[g] > -126 ? __uint_as_float((uint32_t)(e[g] + 126) << 23) : 0.f;
-          lsum += (float)halves * sc;
-        } else {
+        for (int g = 0; g < 2; g++) {
           const float sc = e[g] > -127 ? __uint_as_float((uint32_t)(e[g] + 127) << 23) : 0.f;
           lsum += psum[g] * sc;
         }
+        l = alpha * l + lsum;
       }
-      l = alpha * l + lsum;
 
       if (j > 0) {
         // PV of the previous tile must be done before P is overwritten or O rescaled
@@ -316,6 +394,12 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
 #pragma unroll
             for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(tl + L::T_O + 32 * cc, o);
+          }
+          if (PNQ) {
+            uint32_t lv;
+            tmem_ld1(tl + L::T_O + D, lv);
+            tmem_wait_ld();
+            tmem_st1(tl + L::T_O + D, __float_as_uint(__uint_as_float(lv) * alpha));
           }
           tmem_wait_st();
         }
@@ -344,6 +428,12 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     }
     if (ok) {
       tc_fence_after();
+      if (PNQ) {
+        uint32_t lv;
+        tmem_ld1(tl + L::T_O + D, lv);
+        tmem_wait_ld();
+        l = __uint_as_float(lv);
+      }
       const float inv_l = 1.f / l;
       const int qrow = qt * kBM + row;
       const bool store = qrow < a.N;

@@ -15,6 +15,26 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Named barrier among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also returns the OR of `pred` over the participating threads, so that a
+// decision taken after it (such as leaving a loop) is the same in every participant.
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------------------------------------
 // mbarriers
 // ------------------------------------------------------------------------------------------------
@@ -35,14 +55,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase completes or the hint
+// (nanoseconds) expires, so waiting warps do not take issue slots from working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -181,6 +203,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -218,6 +247,37 @@ __device__ __forceinline__ uint32_t e2m1x32_sum_halves(uint32_t w0, uint32_t w1,
     acc = __dp4a(__byte_perm(kLo, kHi, w[i] >> 16), 0x01010101u, acc);
   }
   return acc;
+}
+
+// max of three fp32 values (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe (no MUFU): Cody-Waite style range reduction
+// x = n + f, n = round(x) via the 1.5 * 2^23 rounding constant, f in [-0.5, 0.5]; 2^f by a
+// degree-5 polynomial (our own minimax fit of 2^f on [-0.5, 0.5], relative error 7.5e-8 before
+// fp32 rounding, 2.2e-7 measured with fp32 Horner evaluation); 2^n added to the exponent
+// field.  Inputs are clamped below at -64 (2^-64 is far below every rounding threshold that
+// matters here); inputs are at most a few units above 0 in the attention kernel.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -64.f);
+  x.y = fmaxf(x.y, -64.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));                         // kRound + n
+  const float2 nn = __ffma2_rn(t, make_float2(-1.f, -1.f), make_float2(kRound, kRound));  // -n
+  const float2 f = __fadd2_rn(x, nn);                                                  // x - n
+  float2 p = __ffma2_rn(make_float2(1.3276472e-3f, 1.3276472e-3f), f, make_float2(9.6755410e-3f, 9.6755410e-3f));
+  p = __ffma2_rn(p, f, make_float2(5.5507131e-2f, 5.5507131e-2f));
+  p = __ffma2_rn(p, f, make_float2(2.4022120e-1f, 2.4022120e-1f));
+  p = __ffma2_rn(p, f, make_float2(6.9314694e-1f, 6.9314694e-1f));
+  p = __ffma2_rn(p, f, make_float2(1.0000001f, 1.0000001f));
+  // the low bits of t hold n; (bits(t) << 23) adds n to the exponent (the constant's own bits
+  // shift out entirely)
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
