@@ -36,7 +36,7 @@ bool make_rule(const mxattn_opts* o, ScaleRule* r) {
   switch (o->scale_rule) {
     case MXATTN_SCALE_UOS: q = 7.25f; break;
     case MXATTN_SCALE_QMAX6: q = 6.0f; break;
-    case MXATTN_SCALE_OCP: r->eq = 2; r->mq = 0xFFFFFFFFu; return true;
+    case MXATTN_SCALE_OCP: r->eq = 2; r->mq = 0xFFFFFFFFu; r->log2q = 2.0f; return true;
     case MXATTN_SCALE_CEIL_CUSTOM:
       q = o->qmax;
       if (!(q >= 4.0f && q <= 8.0f)) return false;  // keeps every exponent inside [-127, 126]
@@ -47,6 +47,7 @@ bool make_rule(const mxattn_opts* o, ScaleRule* r) {
   std::memcpy(&bits, &q, 4);
   r->eq = (int)(bits >> 23) - 127;
   r->mq = bits & 0x007FFFFFu;
+  r->log2q = (float)std::log2((double)q);
   return true;
 }
 

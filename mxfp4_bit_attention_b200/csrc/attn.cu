@@ -46,6 +46,9 @@ constexpr uint32_t kTmemCols = 256;
 // Of the four 8-key words of each 32-key group, this many take their exp2 from the FMA-pipe
 // polynomial instead of MUFU.
 constexpr int kPolyWords = MXATTN_POLY_WORDS;
+#ifndef MXATTN_EXP_LOG2
+#define MXATTN_EXP_LOG2 1
+#endif
 
 template <int D>
 struct Layout {
@@ -100,23 +103,30 @@ __device__ __forceinline__ void raise_abort(volatile int* flag, int* status, int
 }
 
 // Group maximum of 32 raw S values (MASK: keys at index >= valid are excluded).
+#ifndef MXATTN_MAX_CHAINS
+#define MXATTN_MAX_CHAINS 2
+#endif
 template <bool MASK>
 __device__ __forceinline__ float group_max(const uint32_t (&s)[32], int base, int valid) {
-  float a = -INFINITY, b = -INFINITY;
+  constexpr int C = MXATTN_MAX_CHAINS;  // independent max chains
+  float m[C];
 #pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    float v0 = __uint_as_float(s[i]), v1 = __uint_as_float(s[i + 1]);
-    float v2 = __uint_as_float(s[i + 2]), v3 = __uint_as_float(s[i + 3]);
-    if (MASK) {
-      v0 = base + i < valid ? v0 : -INFINITY;
-      v1 = base + i + 1 < valid ? v1 : -INFINITY;
-      v2 = base + i + 2 < valid ? v2 : -INFINITY;
-      v3 = base + i + 3 < valid ? v3 : -INFINITY;
+  for (int k = 0; k < C; k++) m[k] = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2 * C) {
+#pragma unroll
+    for (int k = 0; k < C; k++) {
+      float v0 = __uint_as_float(s[i + 2 * k]), v1 = __uint_as_float(s[i + 2 * k + 1]);
+      if (MASK) {
+        v0 = base + i + 2 * k < valid ? v0 : -INFINITY;
+        v1 = base + i + 2 * k + 1 < valid ? v1 : -INFINITY;
+      }
+      m[k] = fmax3(m[k], v0, v1);
     }
-    a = fmax3(a, v0, v1);
-    b = fmax3(b, v2, v3);
   }
-  return fmaxf(a, b);
+#pragma unroll
+  for (int k = 1; k < C; k++) m[0] = fmaxf(m[0], m[k]);
+  return m[0];
 }
 
 // E2M1 codes of one group of 32: p = 2^(S*c - bias), 4 packed words.  Direct placement also
@@ -150,6 +160,40 @@ __device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, i
     w[q] = cvt_e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
   }
 }
+
+// Phase clock accounting for the diagnostic dump (compiled in only with MXATTN_PHASE_CLOCKS):
+// ck.tick(k) adds the cycles since the previous tick to phase k, in the dumped CTA.
+struct PhaseClock {
+#ifdef MXATTN_PHASE_CLOCKS
+  bool on;
+  long long last;
+  long long acc[8];
+  __device__ __forceinline__ explicit PhaseClock(bool enabled) {
+    on = enabled;
+    last = enabled ? clock64() : 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) acc[i] = 0;
+  }
+  __device__ __forceinline__ void tick(int k) {
+    if (on) {
+      const long long now = clock64();
+      acc[k] += now - last;
+      last = now;
+    }
+  }
+  __device__ __forceinline__ void flush(uint8_t* dump, size_t off, int slot) {
+    if (on) {
+      long long* d = reinterpret_cast<long long*>(dump + off) + slot * 8;
+#pragma unroll
+      for (int i = 0; i < 8; i++) d[i] = acc[i];
+    }
+  }
+#else
+  __device__ __forceinline__ explicit PhaseClock(bool) {}
+  __device__ __forceinline__ void tick(int) {}
+  __device__ __forceinline__ void flush(uint8_t*, size_t, int) {}
+#endif
+};
 
 template <int D, int DT, bool PNQ>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
@@ -357,8 +401,12 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       float bias[2];
 #pragma unroll
       for (int g = 0; g < 2; g++) {
+#if MXATTN_EXP_LOG2
+        e[g] = shared_exponent_log2(gmax[g] == -INFINITY ? -INFINITY : (gmax[g] - sm) * c, a.rule);
+#else
         const float amax = gmax[g] == -INFINITY ? 0.f : ex2_approx((gmax[g] - sm) * c);
         e[g] = shared_exponent(amax, a.rule);
+#endif
         bias[g] = m2 + (float)e[g];
       }
       uint32_t w[8];

@@ -294,7 +294,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
 struct ScaleRule {
   int eq;          // binary exponent of the boundary q
   uint32_t mq;     // its 23 mantissa bits (0xFFFFFFFF: never step up -> floor rule)
+  float log2q;     // fl32(log2 q) for the ceiling rules (unused by the floor rule)
 };
+
+// The same exponent for amax = 2^t given in the log2 domain: ceil(t - log2 q) for the ceiling
+// rules, floor(t) - 2 for the OCP floor rule; clamped to [-127, 127]; t = -inf -> -127.
+// Exact at t = 0 (the group holding the running max: amax = 2^0).
+__device__ __forceinline__ int shared_exponent_log2(float t, ScaleRule r) {
+  if (t == -INFINITY) return -127;
+  int e = r.mq == 0xFFFFFFFFu ? __float2int_rd(t) - 2 : __float2int_ru(t - r.log2q);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
 
 __device__ __forceinline__ int shared_exponent(float amax, ScaleRule r) {
   uint32_t b = __float_as_uint(amax) & 0x7FFFFFFFu;
