@@ -60,11 +60,11 @@ struct Layout {
   static constexpr int STAGE_BYTES = K_BYTES + V_BYTES + ONES_BYTES;
   static constexpr int Q_CODES = 0;
   static constexpr int STAGE0 = Q_BYTES;
-  static constexpr int P_CODES = STAGE0 + kStages * STAGE_BYTES;
   static constexpr int P_BYTES = kBM * kBN / 2;
-  static constexpr int SF_Q = P_CODES + P_BYTES;
-  static constexpr int SF_P = SF_Q + 512;
-  static constexpr int SF_ONES = SF_P + 512;   // scale atom of the ones rows (constant)
+  static constexpr int P_CODES = STAGE0 + kStages * STAGE_BYTES;  // two P buffers
+  static constexpr int SF_Q = P_CODES + 2 * P_BYTES;
+  static constexpr int SF_P = SF_Q + 512;                         // two scale atoms
+  static constexpr int SF_ONES = SF_P + 2 * 512;  // scale atom of the ones rows (constant)
   static constexpr int SF_K = SF_ONES + 512;
   static constexpr int SF_V = SF_K + kStages * 512;
   static constexpr int BARS = SF_V + kStages * 512;
@@ -74,8 +74,8 @@ struct Layout {
     B_KV_EMPTY = 1 + kStages,
     B_S_FULL = 1 + 2 * kStages,
     B_S_FREE,
-    B_P_FULL,
-    B_O_DONE,
+    B_P_FULL,                 // two: one per P buffer
+    B_O_DONE = B_P_FULL + 2,
     B_DRAIN,
     NUM_BARS
   };
@@ -90,8 +90,8 @@ struct Layout {
   static constexpr uint32_t T_S = 0;
   static constexpr uint32_t T_O = 64;                      // O~: D columns, then l at column D
   static constexpr uint32_t T_SFQ = T_O + D + kOnesRows;
-  static constexpr uint32_t T_SFP = T_SFQ + 4;
-  static constexpr uint32_t T_SFK = T_SFP + 4;             // kSfSlots x 4 columns
+  static constexpr uint32_t T_SFP = T_SFQ + 4;             // 2 x 4 columns
+  static constexpr uint32_t T_SFK = T_SFP + 8;             // kSfSlots x 4 columns
   static constexpr uint32_t T_SFV = T_SFK + 4 * kSfSlots;  // kSfSlots x 8 columns (V atom + ones atom)
   static_assert(T_SFV + 8 * kSfSlots <= kTmemCols, "TMEM budget");
   static constexpr uint32_t QK_LAYOUT = D == 128 ? kLayoutSW64 : kLayoutSW32;
@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     mbar_init(bar(L::B_S_FULL), 1);
     mbar_init(bar(L::B_S_FREE), 4);
     mbar_init(bar(L::B_P_FULL), 4);
+    mbar_init(bar(L::B_P_FULL + 1), 4);
     mbar_init(bar(L::B_O_DONE), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     fence_mbar_init();
@@ -292,7 +293,6 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         if (PNQ)
           for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
         const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
-        const uint64_t pdesc = smem_desc(sb + L::P_CODES, 16, 8 * (kBN / 2), kLayoutSW32);
         for (int j = 0; j <= T64; j++) {
           if (j < T64) {
             const int s = j % kStages, f = j % kSfSlots;
@@ -314,6 +314,12 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
               if (!ok) break;
               tc_fence_after();
             }
+            if (j >= 2) {
+              // S(j) also tells the softmax that P buffer j&1 is free: see PV(j-2) complete before
+              // QK(j) is committed (a commit tracks only this thread's work since its last commit)
+              ok = mbar_wait(bar(L::B_O_DONE), (j - 2) & 1, abort_flag, a.wait_budget);
+              if (!ok) break;
+            }
             const uint64_t kdesc = smem_desc(sb + L::STAGE0 + s * L::STAGE_BYTES, 16, 8 * (D / 2), L::QK_LAYOUT);
 #pragma unroll
             for (int kb = 0; kb < D / 64; kb++) {
@@ -326,14 +332,17 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
             mma_commit(bar(L::B_S_FULL));
           }
           if (j > 0) {
-            const int jp = j - 1, sp = jp % kStages, fp = jp % kSfSlots;
-            ok = mbar_wait(bar(L::B_P_FULL), jp & 1, abort_flag, a.wait_budget);
+            const int jp = j - 1, sp = jp % kStages, fp = jp % kSfSlots, pb = jp & 1;
+            ok = mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget);
             if (!ok) break;
             tc_fence_after();
-            tmem_cp_sf_atom(tmem + L::T_SFP, sb + L::SF_P);
+            // P buffer / scale slot pb were last read by PV(jp-2), which this thread saw complete
+            // before committing S(jp); the softmax filled them after S(jp)
+            tmem_cp_sf_atom(tmem + L::T_SFP + 4 * pb, sb + L::SF_P + 512 * pb);
+            const uint64_t pdesc = smem_desc(sb + L::P_CODES + pb * L::P_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
             const uint64_t vdesc =
                 smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
-            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP,
+            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP + 4 * pb,
                      tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
             mma_commit(bar(L::B_O_DONE));
             mma_commit(bar(L::B_KV_EMPTY + sp));
@@ -428,40 +437,40 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         l = alpha * l + lsum;
       }
 
-      if (j > 0) {
-        // PV of the previous tile must be done before P is overwritten or O rescaled
+      // P buffer j&1 was last read by PV(j-2), which the MMA thread saw complete before it
+      // committed the S(j) waited for above.  Only rescaling O~ needs PV(j-1) complete.
+      if (j > 0 && __any_sync(0xFFFFFFFFu, move)) {
         ok = mbar_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.wait_budget);
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xFFFFFFFFu, move)) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; cc++) {
-            uint32_t o[32];
-            tmem_ld32(tl + L::T_O + 32 * cc, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < D / 32; cc++) {
+          uint32_t o[32];
+          tmem_ld32(tl + L::T_O + 32 * cc, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tl + L::T_O + 32 * cc, o);
-          }
-          if (PNQ) {
-            uint32_t lv;
-            tmem_ld1(tl + L::T_O + D, lv);
-            tmem_wait_ld();
-            tmem_st1(tl + L::T_O + D, __float_as_uint(__uint_as_float(lv) * alpha));
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tl + L::T_O + 32 * cc, o);
         }
+        if (PNQ) {
+          uint32_t lv;
+          tmem_ld1(tl + L::T_O + D, lv);
+          tmem_wait_ld();
+          tmem_st1(tl + L::T_O + D, __float_as_uint(__uint_as_float(lv) * alpha));
+        }
+        tmem_wait_st();
       }
-      uint8_t* prow = smem + L::P_CODES + row * (kBN / 2);
+      const int pb = j & 1;
+      uint8_t* prow = smem + L::P_CODES + pb * L::P_BYTES + row * (kBN / 2);
       const int sw = (row >> 2) & 1;
       *reinterpret_cast<uint4*>(prow + (sw * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       *reinterpret_cast<uint4*>(prow + ((1 ^ sw) * 16)) = make_uint4(w[4], w[5], w[6], w[7]);
-      *reinterpret_cast<uint16_t*>(smem + L::SF_P + (row % 32) * 16 + (row / 32) * 4) =
+      *reinterpret_cast<uint16_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
           (uint16_t)((e[0] + 127) | ((e[1] + 127) << 8));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_P_FULL));
+      if (lane == 0) mbar_arrive(bar(L::B_P_FULL + pb));
       if (dumping) {
         uint32_t* dp = reinterpret_cast<uint32_t*>(a.dump + dl.p_codes + ((size_t)j * 128 + row) * 32);
         for (int i = 0; i < 8; i++) dp[i] = w[i];
