@@ -214,9 +214,7 @@ def dump_layout(N: int, d: int) -> dict:
     o = (p_scales + T64 * 128 * 2 + 15) // 16 * 16
     l = o + 128 * d * 4
     m = l + 128 * 4
-    clocks = (m + 128 * 4 + 15) // 16 * 16
-    return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "clocks": clocks,
-            "total": clocks + 192 * 8 * 8}
+    return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "total": m + 128 * 4}
 
 
 def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, dump_qt=0, opts=None,
@@ -246,8 +244,7 @@ def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, 
             "p_scales": raw[L["p_scales"]:L["p_scales"] + T64 * 256].reshape(T64, 128, 2),
             "o": raw[L["o"]:L["l"]].view(np.float32).reshape(128, d),
             "l": raw[L["l"]:L["m"]].view(np.float32).copy(),
-            "m": raw[L["m"]:L["m"] + 512].view(np.float32).copy(),
-            "clocks": raw[L["clocks"]:L["total"]].view(np.int64).reshape(192, 8).copy()}
+            "m": raw[L["m"]:L["m"] + 512].view(np.float32).copy()}
 
 
 def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None, stream=None):

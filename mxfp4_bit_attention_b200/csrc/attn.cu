@@ -9,8 +9,9 @@
 // One CTA owns 128 query rows of one head and sweeps all keys in tiles of 64:
 //   warp 4 (one lane)  bulk-copies Q^ once and K^/V^ tiles + their scale atoms into a
 //                      4-stage shared-memory ring;
-//   warp 5 (one lane)  issues tcgen05.mma kind::mxf4 block-scaled MMAs:
-//                      S = Q^ K^T (TMEM, fp32) and O~ += P^ V^ (TMEM, fp32);
+//   warp 5             issues S = Q^ K^T (tcgen05.mma kind::mxf4 block-scaled, fp32 in TMEM);
+//   warp 6             issues O~ += P^ V^ (same kind, fp32 in TMEM); the two issuers split the
+//                      serial per-tile cost of tcgen05 issue and mbarrier waits;
 //   warps 0-3          one query row per thread: read S from TMEM, online max (optionally lazy,
 //                      threshold tau in log2 units), P~ = 2^(S*c - m) folded with the MXFP4 scale
 //                      of each 32-key group, E2M1 codes of P~ written to shared memory in the
@@ -37,7 +38,10 @@ constexpr int kBM = 128;        // query rows per CTA
 constexpr int kBN = 64;         // keys per tile
 constexpr int kStages = 4;      // K/V shared-memory ring depth
 constexpr int kSfSlots = 3;     // K/V scale-factor slots in TMEM (reuse distance 3 tiles)
-constexpr int kThreads = 192;   // 4 softmax warps, producer warp, MMA warp
+constexpr int kThreads = 224;   // 4 softmax warps, producer warp, QK and PV MMA issuer warps
+constexpr int kProducerWarp = 4;
+constexpr int kQkWarp = 5;
+constexpr int kPvWarp = 6;
 constexpr int kOnesRows = 16;   // rows appended to V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 256;
 #ifndef MXATTN_POLY_WORDS
@@ -46,9 +50,6 @@ constexpr uint32_t kTmemCols = 256;
 // Of the four 8-key words of each 32-key group, this many take their exp2 from the FMA-pipe
 // polynomial instead of MUFU.
 constexpr int kPolyWords = MXATTN_POLY_WORDS;
-#ifndef MXATTN_EXP_LOG2
-#define MXATTN_EXP_LOG2 1
-#endif
 
 template <int D>
 struct Layout {
@@ -75,8 +76,8 @@ struct Layout {
     B_S_FULL = 1 + 2 * kStages,
     B_S_FREE,
     B_P_FULL,                 // two: one per P buffer
-    B_O_DONE = B_P_FULL + 2,
-    B_DRAIN,
+    B_O_DONE = B_P_FULL + 2,  // two: PV MMAs of even and odd tiles
+    B_DRAIN = B_O_DONE + 2,
     NUM_BARS
   };
   static constexpr int TMEM_SLOT = BARS + NUM_BARS * 8;
@@ -161,40 +162,6 @@ __device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, i
   }
 }
 
-// Phase clock accounting for the diagnostic dump (compiled in only with MXATTN_PHASE_CLOCKS):
-// ck.tick(k) adds the cycles since the previous tick to phase k, in the dumped CTA.
-struct PhaseClock {
-#ifdef MXATTN_PHASE_CLOCKS
-  bool on;
-  long long last;
-  long long acc[8];
-  __device__ __forceinline__ explicit PhaseClock(bool enabled) {
-    on = enabled;
-    last = enabled ? clock64() : 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) acc[i] = 0;
-  }
-  __device__ __forceinline__ void tick(int k) {
-    if (on) {
-      const long long now = clock64();
-      acc[k] += now - last;
-      last = now;
-    }
-  }
-  __device__ __forceinline__ void flush(uint8_t* dump, size_t off, int slot) {
-    if (on) {
-      long long* d = reinterpret_cast<long long*>(dump + off) + slot * 8;
-#pragma unroll
-      for (int i = 0; i < 8; i++) d[i] = acc[i];
-    }
-  }
-#else
-  __device__ __forceinline__ explicit PhaseClock(bool) {}
-  __device__ __forceinline__ void tick(int) {}
-  __device__ __forceinline__ void flush(uint8_t*, size_t, int) {}
-#endif
-};
-
 template <int D, int DT, bool PNQ>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
   using L = Layout<D>;
@@ -224,7 +191,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     mbar_init(bar(L::B_P_FULL), 4);
     mbar_init(bar(L::B_P_FULL + 1), 4);
     mbar_init(bar(L::B_O_DONE), 1);
-    mbar_init(bar(L::B_DRAIN), 1);
+    mbar_init(bar(L::B_O_DONE + 1), 1);
+    mbar_init(bar(L::B_DRAIN), 2);  // one commit from each issuer
     fence_mbar_init();
   }
   if (PNQ) {
@@ -239,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       reinterpret_cast<uint32_t*>(smem + L::SF_ONES)[i] = i == 0 ? 0x7F7F7F7Fu : 0u;
     fence_proxy_async_smem();
   }
-  if (warp == 5) {
+  if (warp == kQkWarp) {
     tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
     tmem_relinquish();
   }
@@ -249,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::TMEM_SLOT);
   const volatile int* no_abort = &never;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
@@ -283,77 +251,98 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           mbar_wait(bar(L::B_KV_FULL + j % kStages), (j / kStages) & 1, no_abort, a.wait_budget);
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget);
-      if (ok) {
+  } else if (warp == kQkWarp) {
+    // ------------------------------------------------------------------ QK issuer
+    // The warp runs the loop converged (waits and descriptor arithmetic stay warp-uniform); lane 0
+    // alone issues its tcgen05 operations, so that each of its commits covers all of them.
+    const bool leader = lane == 0;
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget));
+    if (ok) {
+      tc_fence_after();
+      if (leader) tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
+      __syncwarp();
+      const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
+      for (int j = 0; j < T64; j++) {
+        const int s = j % kStages, f = j % kSfSlots;
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
+        if (!ok) break;
         tc_fence_after();
-        tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
-        if (PNQ)
-          for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
-        const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
-        for (int j = 0; j <= T64; j++) {
-          if (j < T64) {
-            const int s = j % kStages, f = j % kSfSlots;
-            ok = mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget);
-            if (!ok) break;
-            tc_fence_after();
-            if (PNQ && D == 64) {
-              // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
-              // channels >= d are zero): give it scale 2^0 for all four key groups
-              *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * s + 8) = 0x7F7F7F7Fu;
-              fence_proxy_async_smem();
-            }
-            // slot f was last read by the MMAs of tile j-3, complete since the softmax saw
-            // O_DONE(j-3) before releasing P(j-2), which this thread waited for
-            tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
-            tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f, sb + L::SF_V + 512 * s);
-            if (j > 0) {
-              ok = mbar_wait(bar(L::B_S_FREE), (j - 1) & 1, abort_flag, a.wait_budget);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            if (j >= 2) {
-              // S(j) also tells the softmax that P buffer j&1 is free: see PV(j-2) complete before
-              // QK(j) is committed (a commit tracks only this thread's work since its last commit)
-              ok = mbar_wait(bar(L::B_O_DONE), (j - 2) & 1, abort_flag, a.wait_budget);
-              if (!ok) break;
-            }
-            const uint64_t kdesc = smem_desc(sb + L::STAGE0 + s * L::STAGE_BYTES, 16, 8 * (D / 2), L::QK_LAYOUT);
-#pragma unroll
-            for (int kb = 0; kb < D / 64; kb++) {
-              // K block kb covers head dims 64kb..64kb+63: 32 bytes further along each row,
-              // scale bytes 2kb and 2kb+1 of each row's scale word.
-              mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
-                       mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
-                       tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(L::B_S_FULL));
-          }
-          if (j > 0) {
-            const int jp = j - 1, sp = jp % kStages, fp = jp % kSfSlots, pb = jp & 1;
-            ok = mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget);
-            if (!ok) break;
-            tc_fence_after();
-            // P buffer / scale slot pb were last read by PV(jp-2), which this thread saw complete
-            // before committing S(jp); the softmax filled them after S(jp)
-            tmem_cp_sf_atom(tmem + L::T_SFP + 4 * pb, sb + L::SF_P + 512 * pb);
-            const uint64_t pdesc = smem_desc(sb + L::P_CODES + pb * L::P_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
-            const uint64_t vdesc =
-                smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
-            mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP + 4 * pb,
-                     tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
-            mma_commit(bar(L::B_O_DONE));
-            mma_commit(bar(L::B_KV_EMPTY + sp));
-          }
+        // K scale slot f was last read by QK(j-3), complete since the softmax read S(j-3)
+        // before releasing it, which this warp waited for
+        if (leader) tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
+        if (j > 0) {
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_S_FREE), (j - 1) & 1, abort_flag, a.wait_budget));
+          if (!ok) break;
+          tc_fence_after();
         }
+        if (j >= 2) {
+          // S(j) also tells the softmax that P buffer j&1 (last read by PV(j-2)) is free: see
+          // PV(j-2) complete first.  Each O_DONE barrier is at most one phase away from it.
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget));
+          if (!ok) break;
+        }
+        const uint64_t kdesc = smem_desc(sb + L::STAGE0 + s * L::STAGE_BYTES, 16, 8 * (D / 2), L::QK_LAYOUT);
+        if (leader) {
+#pragma unroll
+          for (int kb = 0; kb < D / 64; kb++) {
+            // K block kb covers head dims 64kb..64kb+63: 32 bytes further along each row,
+            // scale bytes 2kb and 2kb+1 of each row's scale word.
+            mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
+                     mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
+                     tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_S_FULL));
+        }
+        __syncwarp();
       }
-      if (!ok) raise_abort(abort_flag, a.status, 2);
-      // wait for every tcgen05 operation this thread issued before TMEM is released
-      mma_commit(bar(L::B_DRAIN));
-      mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
     }
+    if (!ok && leader) raise_abort(abort_flag, a.status, 2);
+    // wait for every tcgen05 operation of both issuers before TMEM is released
+    if (leader) mma_commit(bar(L::B_DRAIN));
+    __syncwarp();
+    mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------------ PV issuer (same scheme)
+    const bool leader = lane == 0;
+    if (PNQ && leader)
+      for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
+    __syncwarp();
+    bool ok = true;
+    for (int jp = 0; jp < T64; jp++) {
+      const int sp = jp % kStages, fp = jp % kSfSlots, pb = jp & 1;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget));
+      if (!ok) break;
+      // V^(jp) landed with K^(jp), before S(jp) and so before P(jp); this warp also waits for the
+      // stage itself (it cannot have been refilled: that needs this warp's commit below)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + sp), (jp / kStages) & 1, abort_flag, a.wait_budget));
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t pdesc = smem_desc(sb + L::P_CODES + pb * L::P_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
+      const uint64_t vdesc =
+          smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
+      if (leader) {
+        // P scale slot pb and V scale slot fp were last read by PV(jp-2) and PV(jp-3), complete
+        // before S(jp) was committed, which the softmax saw before writing P(jp)
+        tmem_cp_sf_atom(tmem + L::T_SFP + 4 * pb, sb + L::SF_P + 512 * pb);
+        if (PNQ && D == 64) {
+          // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
+          // channels >= d are zero): give it scale 2^0 for all four key groups
+          *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * sp + 8) = 0x7F7F7F7Fu;
+          fence_proxy_async_smem();
+        }
+        tmem_cp_sf_atom(tmem + L::T_SFV + 8 * fp, sb + L::SF_V + 512 * sp);
+        mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP + 4 * pb,
+                 tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
+        mma_commit(bar(L::B_O_DONE + (jp & 1)));
+        // QK(jp) read the stage too: complete, since the softmax saw S(jp) before P(jp)
+        mma_commit(bar(L::B_KV_EMPTY + sp));
+      }
+      __syncwarp();
+    }
+    if (!ok && leader) raise_abort(abort_flag, a.status, 4);
+    if (leader) mma_commit(bar(L::B_DRAIN));
+    __syncwarp();
+    mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
   } else {
     // ------------------------------------------------------------------ softmax (warps 0-3)
     const int row = threadIdx.x;  // TMEM lane and query row within the tile
@@ -399,25 +388,20 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       // max, as exp(0) is in the oracle, so scale rules whose boundaries sit on powers of two
       // (OCP, q = 4 or 8) decide it the same way.
       const float mt_raw = fmaxf(gmax[0], gmax[1]);
-      const bool first = (j == 0);
-      const bool move = first || (mt_raw * c > m2 + a.tau);
-      const float sm_new = move ? mt_raw : sm;
-      const float alpha = first ? 0.f : (move ? ex2_approx((sm - sm_new) * c) : 1.f);
-      sm = sm_new;
+      const bool move = j == 0 || (mt_raw * c > m2 + a.tau);
+      // O~ and l are rescaled by alpha = 2^(m_old - m_new) only when some row of the warp moves
+      // its max (alpha = 1 elsewhere); tile 0 starts both at zero
+      const bool any_move = j > 0 && __any_sync(0xFFFFFFFFu, move);
+      const float sm_old = sm;
+      if (move) sm = mt_raw;
       m2 = sm * c;
+      float alpha = 1.f;
+      if (any_move && move) alpha = ex2_approx((sm_old - sm) * c);
 
-      int e[2];
+      uint32_t eb[2];  // E8M0 bytes
       float bias[2];
 #pragma unroll
-      for (int g = 0; g < 2; g++) {
-#if MXATTN_EXP_LOG2
-        e[g] = shared_exponent_log2(gmax[g] == -INFINITY ? -INFINITY : (gmax[g] - sm) * c, a.rule);
-#else
-        const float amax = gmax[g] == -INFINITY ? 0.f : ex2_approx((gmax[g] - sm) * c);
-        e[g] = shared_exponent(amax, a.rule);
-#endif
-        bias[g] = m2 + (float)e[g];
-      }
+      for (int g = 0; g < 2; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);
       uint32_t w[8];
       float psum[2] = {0.f, 0.f};
       if (full) {
@@ -430,17 +414,14 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       if (!PNQ) {
         float lsum = 0.f;
 #pragma unroll
-        for (int g = 0; g < 2; g++) {
-          const float sc = e[g] > -127 ? __uint_as_float((uint32_t)(e[g] + 127) << 23) : 0.f;
-          lsum += psum[g] * sc;
-        }
+        for (int g = 0; g < 2; g++) lsum += psum[g] * __uint_as_float(eb[g] << 23);  // byte 0: 2^-127 -> 0
         l = alpha * l + lsum;
       }
 
-      // P buffer j&1 was last read by PV(j-2), which the MMA thread saw complete before it
-      // committed the S(j) waited for above.  Only rescaling O~ needs PV(j-1) complete.
-      if (j > 0 && __any_sync(0xFFFFFFFFu, move)) {
-        ok = mbar_wait(bar(L::B_O_DONE), (j - 1) & 1, abort_flag, a.wait_budget);
+      // Rescaling O~ needs PV(j-1) complete.  Each O_DONE barrier (even / odd tiles) can be at
+      // most one phase behind or ahead of the phase waited for here.
+      if (any_move) {
+        ok = mbar_wait(bar(L::B_O_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, a.wait_budget);
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
@@ -460,13 +441,15 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
         tmem_wait_st();
       }
+      // P buffer pb was last read by PV(j-2), which the QK issuer saw complete before it
+      // committed S(j)
       const int pb = j & 1;
       uint8_t* prow = smem + L::P_CODES + pb * L::P_BYTES + row * (kBN / 2);
       const int sw = (row >> 2) & 1;
       *reinterpret_cast<uint4*>(prow + (sw * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       *reinterpret_cast<uint4*>(prow + ((1 ^ sw) * 16)) = make_uint4(w[4], w[5], w[6], w[7]);
       *reinterpret_cast<uint16_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
-          (uint16_t)((e[0] + 127) | ((e[1] + 127) << 8));
+          (uint16_t)(eb[0] | (eb[1] << 8));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -475,12 +458,16 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         uint32_t* dp = reinterpret_cast<uint32_t*>(a.dump + dl.p_codes + ((size_t)j * 128 + row) * 32);
         for (int i = 0; i < 8; i++) dp[i] = w[i];
         uint8_t* dsf = a.dump + dl.p_scales + ((size_t)j * 128 + row) * 2;
-        dsf[0] = (uint8_t)(e[0] + 127);
-        dsf[1] = (uint8_t)(e[1] + 127);
+        dsf[0] = (uint8_t)eb[0];
+        dsf[1] = (uint8_t)eb[1];
       }
     }
+    if (ok && T64 >= 2) {  // the last two PV MMAs, one on each O_DONE barrier
+      ok = mbar_wait(bar(L::B_O_DONE + (T64 & 1)), ((T64 - 2) >> 1) & 1, abort_flag, a.wait_budget);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+    }
     if (ok) {
-      ok = mbar_wait(bar(L::B_O_DONE), (T64 - 1) & 1, abort_flag, a.wait_budget);
+      ok = mbar_wait(bar(L::B_O_DONE + ((T64 - 1) & 1)), ((T64 - 1) >> 1) & 1, abort_flag, a.wait_budget);
       ok = __all_sync(0xFFFFFFFFu, ok);
     }
     if (ok) {
@@ -537,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kQkWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

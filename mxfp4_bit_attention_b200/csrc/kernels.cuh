@@ -65,11 +65,8 @@ struct AttnArgs {
 //   P scales               [T64][128][2] bytes (E8M0 of key groups 0 and 1 of the tile)
 //   O accumulator          [128][D] fp32, before the division by l
 //   l, m                   [128] fp32 each (m in log2 units: running max of S * scale * log2 e)
-//   phase clocks           [192][8] int64: per thread, SM clock cycles summed over all tiles
-//                          for each phase of its role (softmax rows 0..127, producer 128,
-//                          MMA issuer 160; see the kernel for the phase numbering)
 struct DumpLayout {
-  size_t s, p_codes, p_scales, o, l, m, clocks, total;
+  size_t s, p_codes, p_scales, o, l, m, total;
   __host__ __device__ DumpLayout(int D, int T64) {
     s = 0;
     p_codes = 2 * 128 * 64 * 4;
@@ -77,8 +74,7 @@ struct DumpLayout {
     o = (p_scales + (size_t)T64 * 128 * 2 + 15) / 16 * 16;
     l = o + (size_t)128 * D * 4;
     m = l + 128 * 4;
-    clocks = (m + 128 * 4 + 15) / 16 * 16;
-    total = clocks + 192 * 8 * 8;
+    total = m + 128 * 4;
   }
 };
 

@@ -55,17 +55,40 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// try_wait with a suspend-time hint: the thread sleeps until the phase completes or the hint
-// (nanoseconds) expires, so waiting warps do not take issue slots from working ones.
+// try_wait: the thread may sleep until the phase completes or a time limit passes, so waiting
+// warps do not take issue slots from working ones.  MXATTN_WAIT_HINT_NS > 0 passes that limit
+// (nanoseconds) as a suspend-time hint; 0 (the default, measured fastest here) leaves it to the
+// hardware; < 0 selects the non-blocking test_wait, for experiments.
+#ifndef MXATTN_WAIT_HINT_NS
+#define MXATTN_WAIT_HINT_NS 0
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+#if MXATTN_WAIT_HINT_NS > 0
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(1000000u)
+      : "r"(bar), "r"(parity), "r"((uint32_t)MXATTN_WAIT_HINT_NS)
       : "memory");
+#elif MXATTN_WAIT_HINT_NS == 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+#else  // negative: non-blocking test, the caller spins
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+#endif
   return ok != 0;
 }
 
@@ -297,13 +320,23 @@ struct ScaleRule {
   float log2q;     // fl32(log2 q) for the ceiling rules (unused by the floor rule)
 };
 
-// The same exponent for amax = 2^t given in the log2 domain: ceil(t - log2 q) for the ceiling
-// rules, floor(t) - 2 for the OCP floor rule; clamped to [-127, 127]; t = -inf -> -127.
-// Exact at t = 0 (the group holding the running max: amax = 2^0).
-__device__ __forceinline__ int shared_exponent_log2(float t, ScaleRule r) {
-  if (t == -INFINITY) return -127;
-  int e = r.mq == 0xFFFFFFFFu ? __float2int_rd(t) - 2 : __float2int_ru(t - r.log2q);
-  return e < -127 ? -127 : (e > 127 ? 127 : e);
+// shared_exponent for amax = 2^t given in the log2 domain: ceil(t - log2 q) for the ceiling
+// rules, floor(t) - 2 for the OCP floor rule, clamped to [-127, 127] (exact at t = 0, the group
+// holding the running max).  Computed on the FMA pipe alone and returned as an exact float,
+// with its E8M0 byte (e + 127).  Adding x to M = 1.5 * 2^23 + 127 with rounding toward +inf
+// (ceiling rules) or -inf (floor rule) lands on the integer M + ceil(x) or M + floor(x), in a
+// binade whose ulp is 1, so the sum's low mantissa bits are 127 + e.  Clamping x to
+// [-127, 127] first (an integer range) clamps e the same way; t = -inf gives -127.
+__device__ __forceinline__ float shared_exponent_log2f(float t, ScaleRule r, uint32_t& byte) {
+  constexpr float M = 12582912.f + 127.f;
+  float y;
+  if (r.mq == 0xFFFFFFFFu) {  // floor(t) - 2: floor t itself (t - 2 could round), M - 2 adds the -2
+    y = __fadd_rd(fminf(fmaxf(t, -125.f), 129.f), M - 2.f);
+  } else {
+    y = __fadd_ru(fminf(fmaxf(t - r.log2q, -127.f), 127.f), M);
+  }
+  byte = __float_as_uint(y) & 0xFFu;
+  return y - M;
 }
 
 __device__ __forceinline__ int shared_exponent(float amax, ScaleRule r) {
