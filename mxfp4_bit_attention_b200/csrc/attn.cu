@@ -38,14 +38,29 @@ constexpr int kBM = 128;        // query rows per CTA
 constexpr int kBN = 64;         // keys per tile
 constexpr int kStages = 4;      // K/V shared-memory ring depth
 constexpr int kSfSlots = 3;     // K/V scale-factor slots in TMEM (reuse distance 3 tiles)
-constexpr int kThreads = 224;   // 4 softmax warps, producer warp, QK and PV MMA issuer warps
-constexpr int kProducerWarp = 4;
-constexpr int kQkWarp = 5;
-constexpr int kPvWarp = 6;
+// Warps 0-3 run the softmax (warp w reads TMEM lanes 32w..32w+31); the producer and the two MMA
+// issuers take three of the warps after them (where they sit was measured not to matter).
+#ifndef MXATTN_PRODUCER_WARP
+#define MXATTN_PRODUCER_WARP 4
+#endif
+#ifndef MXATTN_QK_WARP
+#define MXATTN_QK_WARP 5
+#endif
+#ifndef MXATTN_PV_WARP
+#define MXATTN_PV_WARP 6
+#endif
+constexpr int kProducerWarp = MXATTN_PRODUCER_WARP;
+constexpr int kQkWarp = MXATTN_QK_WARP;
+constexpr int kPvWarp = MXATTN_PV_WARP;
+constexpr int kWarps = 1 + (kProducerWarp > kQkWarp ? (kProducerWarp > kPvWarp ? kProducerWarp : kPvWarp)
+                                                    : (kQkWarp > kPvWarp ? kQkWarp : kPvWarp));
+constexpr int kThreads = 32 * kWarps;  // 224 with the default roles
+static_assert(kProducerWarp >= 4 && kQkWarp >= 4 && kPvWarp >= 4 && kProducerWarp != kQkWarp &&
+                  kProducerWarp != kPvWarp && kQkWarp != kPvWarp, "warp roles");
 constexpr int kOnesRows = 16;   // rows appended to V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 256;
 #ifndef MXATTN_POLY_WORDS
-#define MXATTN_POLY_WORDS 0
+#define MXATTN_POLY_WORDS 1
 #endif
 // Of the four 8-key words of each 32-key group, this many take their exp2 from the FMA-pipe
 // polynomial instead of MUFU.
@@ -343,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     if (leader) mma_commit(bar(L::B_DRAIN));
     __syncwarp();
     mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------------ softmax (warps 0-3)
     const int row = threadIdx.x;  // TMEM lane and query row within the tile
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
@@ -354,14 +369,19 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     float m2 = -INFINITY;  // the same in log2 units, fl32(sm * c)
     float l = 0.f;         // direct placement only (PNQ keeps l in O~ column D)
     bool ok = true;
+    bool s_ready = false;  // S(j) was seen complete by the early test during tile j-1
     for (int j = 0; j < T64; j++) {
-      ok = mbar_wait(bar(L::B_S_FULL), j & 1, abort_flag, a.wait_budget);
-      if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+      if (!__all_sync(0xFFFFFFFFu, s_ready)) {
+        ok = mbar_wait(bar(L::B_S_FULL), j & 1, abort_flag, a.wait_budget);
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+      }
       tc_fence_after();
       uint32_t s0[32], s1[32];
       tmem_ld32(tl + L::T_S, s0);
       tmem_ld32(tl + L::T_S + 32, s1);
       tmem_wait_ld();
+      pin32(s0);
+      pin32(s1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_S_FREE));
@@ -411,6 +431,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         group_codes<true, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
         group_codes<true, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
       }
+      // test S(j+1) now, so that the test's latency overlaps the stores below
+      s_ready = j + 1 < T64 && mbar_test(bar(L::B_S_FULL), (j + 1) & 1);
       if (!PNQ) {
         float lsum = 0.f;
 #pragma unroll
@@ -429,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           uint32_t o[32];
           tmem_ld32(tl + L::T_O + 32 * cc, o);
           tmem_wait_ld();
+          pin32(o);
 #pragma unroll
           for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tl + L::T_O + 32 * cc, o);
@@ -437,6 +460,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           uint32_t lv;
           tmem_ld1(tl + L::T_O + D, lv);
           tmem_wait_ld();
+          pin1(lv);
           tmem_st1(tl + L::T_O + D, __float_as_uint(__uint_as_float(lv) * alpha));
         }
         tmem_wait_st();
@@ -476,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         uint32_t lv;
         tmem_ld1(tl + L::T_O + D, lv);
         tmem_wait_ld();
+        pin1(lv);
         l = __uint_as_float(lv);
       }
       const float inv_l = 1.f / l;
@@ -487,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         uint32_t o[32];
         tmem_ld32(tl + L::T_O + 32 * cc, o);
         tmem_wait_ld();
+        pin32(o);
         if (dumping) {
           float* d_o = reinterpret_cast<float*>(a.dump + dl.o) + (size_t)row * D + 32 * cc;
           for (int i = 0; i < 32; i++) d_o[i] = __uint_as_float(o[i]);

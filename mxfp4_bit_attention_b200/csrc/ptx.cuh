@@ -92,6 +92,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase: true once it has completed (with the same acquire semantics as
+// a successful try_wait).  Its result is only needed when the caller branches on it, so a test
+// issued early overlaps its latency with other work.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait.  Gives up (returns false) after `budget` SM clock cycles, or as
 // soon as *abort becomes non-zero (another warp gave up first).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
@@ -234,6 +249,15 @@ __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Registers filled by tcgen05.ld hold their values only after tcgen05.wait::ld.  These empty
+// volatile asm statements, placed after the wait, make every later use of the registers depend
+// on a point after it, so the compiler cannot move a use above the wait.
+__device__ __forceinline__ void pin1(uint32_t& r) { asm volatile("" : "+r"(r)); }
+__device__ __forceinline__ void pin32(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i++) pin1(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------------------------------------
