@@ -73,7 +73,7 @@ def lib():
             L.mxref_dequantize.argtypes = [P, P, i64, P]
             L.mxref_dequantize.restype = None
             L.mxref_attention_rows.argtypes = [P, i64, P, P, i32, i32, f32, ctypes.POINTER(AttnCfg),
-                                               P, P, P, P, P]
+                                               P, P, P, P, P, P, P]
             L.mxref_attention_rows.restype = None
             L.mxref_num_threads.argtypes = []
             L.mxref_num_threads.restype = i32
@@ -160,9 +160,10 @@ def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------------------------
 
 def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=True, rule=RULE_UOS,
-                   qmax=7.25, tau=0.0, weights=False):
+                   qmax=7.25, tau=0.0, weights=False, codes=False):
     """Online-softmax attention with PNQ for query rows qd [n, d] against
-    kd, vd [N, d] (fp64 values).  Returns dict(out, m, l[, wsum, ocheck])."""
+    kd, vd [N, d] (fp64 values).  Returns dict(out, m, l[, wsum, ocheck]
+    [, p_codes [n, ntiles*key_tile], p_scales [n, ntiles*key_tile/32]])."""
     qd = np.ascontiguousarray(qd, dtype=np.float64)
     kd = np.ascontiguousarray(kd, dtype=np.float64)
     vd = np.ascontiguousarray(vd, dtype=np.float64)
@@ -175,9 +176,16 @@ def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=Tru
     l = np.empty(n, np.float64)
     wsum = np.empty(n, np.float64) if weights else None
     ocheck = np.empty((n, d), np.float64) if weights else None
+    ntiles = (N + key_tile - 1) // key_tile
+    pc = np.zeros((n, ntiles * key_tile), np.uint8) if codes else None
+    ps = np.zeros((n, ntiles * key_tile // 32), np.uint8) if codes else None
     lib().mxref_attention_rows(_ptr(qd), n, _ptr(kd), _ptr(vd), N, d, float(np.float32(softmax_scale)),
-                               ctypes.byref(cfg), _ptr(out), _ptr(m), _ptr(l), _ptr(wsum), _ptr(ocheck))
+                               ctypes.byref(cfg), _ptr(out), _ptr(m), _ptr(l), _ptr(wsum), _ptr(ocheck),
+                               _ptr(pc), _ptr(ps))
     res = {"out": out, "m": m, "l": l}
+    if codes:
+        res["p_codes"] = pc
+        res["p_scales"] = ps
     if weights:
         res["wsum"] = wsum
         res["ocheck"] = ocheck

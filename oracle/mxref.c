@@ -255,10 +255,14 @@ typedef struct {
  * w_k = P^_k * prod(alpha of the later tiles) / l, accumulated key by key
  * independently of the l recurrence, and ocheck [nrows][d] = sum_k w_k v_k,
  * the output rebuilt from those weights (both need wsum and ocheck non-NULL).
+ * pcodes [nrows][ntiles*T] and pscales [nrows][ntiles*T/32], when non-NULL,
+ * receive the E2M1 codes (one per byte, keys in order, padded keys 0) and the
+ * E8M0 scale bytes of every quantized P~ group (quant_p only).
  */
 void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const double* v, int N,
                           int d, float scale, const mxref_attn_cfg* cfg, double* out, double* m_out,
-                          double* l_out, double* wsum_out, double* ocheck_out) {
+                          double* l_out, double* wsum_out, double* ocheck_out, uint8_t* pcodes_out,
+                          uint8_t* pscales_out) {
   const int T = cfg->key_tile;
   const int ntiles = (N + T - 1) / T;
 #pragma omp parallel
@@ -297,6 +301,8 @@ void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const
           for (int g = 0; g < T / 32; g++) {
             int sb = quantize_group(pt + g * 32, 32, 1, cfg->rule, cfg->qmax, codes);
             for (int i = 0; i < 32; i++) ph[g * 32 + i] = ldexp(mxref_e2m1_decode(codes[i]), sb - 127);
+            if (pcodes_out) memcpy(pcodes_out + ((size_t)r * ntiles + t) * T + g * 32, codes, 32);
+            if (pscales_out) pscales_out[((size_t)r * ntiles + t) * (T / 32) + g] = (uint8_t)sb;
           }
         } else {
           for (int j = 0; j < T; j++) ph[j] = (double)pt[j];

@@ -102,3 +102,20 @@ def test_rows_are_independent(tiny):
     full = oracle.forward_rows(q[None], k[None], v[None], np.arange(256), 0.125)
     part = oracle.forward_rows(q[None], k[None], v[None], rows, 0.125)
     assert np.array_equal(full["out"][0][rows], part["out"][0])
+
+
+@pytest.mark.parametrize("N", [64, 45])
+def test_recorded_p_codes_rebuild_the_pnq_row_sum(tiny, N):
+    """With one key tile there is no rescaling, so under PNQ the row sum l is exactly the sum of
+    the quantized tile: the recorded codes and scale bytes, dequantized, must rebuild it; keys
+    past N (ragged tile) must record code 0, and each group's largest value must sit on the
+    E2M1 grid scaled by its recorded power of two."""
+    q, k, v = (x.astype(np.float64) for x in tiny)
+    r = oracle.attention_rows(q[:16], k[:N], v[:N], 0.125, tau=0.0, codes=True)
+    pc, ps = r["p_codes"], r["p_scales"]
+    assert pc.shape == (16, 64) and ps.shape == (16, 2)
+    assert not pc[:, N:].any()
+    vals = oracle.dequantize(pc, ps)
+    np.testing.assert_allclose(vals.sum(axis=1), r["l"], rtol=1e-15, atol=0)
+    # the group holding the row max (P~ = exp(0) = 1) is never all zero
+    assert (vals.max(axis=1) > 0).all()
