@@ -156,13 +156,26 @@ def dist_setup(n_gpus: int):
     return rank, world, dist
 
 
-def reduce_max(x: float, dist) -> float:
+def reduce_max(x: float, dist, device: str = "cuda") -> float:
+    """Max of a per-rank timing over all ranks (the job's time is its slowest rank's)."""
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Batch element `rank` of a B = world batch: the workload's shape with its own seeded inputs.
+    The ranks' problems are independent, so no data moves between GPUs."""
+    from mxfp4_bit_attention_b200 import inputs
+    return inputs.Workload(w.name, 1, w.H, w.N, w.d, w.dtype, w.seed + 1000 * rank)
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Throughput of the whole job: every rank's flops over the slowest rank's step time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
 def barrier(dist):
@@ -244,8 +257,7 @@ def main():
     binding.load()
 
     # inputs: batch element `rank` of a B = world batch (independent problems)
-    wl = inputs.Workload(w.name, 1, w.H, w.N, w.d, w.dtype, w.seed + 1000 * rank)
-    g = inputs.generate(wl)
+    g = inputs.generate(rank_workload(w, rank))
     shape = (1, w.H, w.N, w.d)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
@@ -305,7 +317,7 @@ def main():
     attn_ms_max = reduce_max(attn_ms, dist)
     ms_per_step = total_ms / args.steps
     flops = w.flops  # per rank (B = 1 per rank)
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, ms_per_step)
     clocks = clk.summary()
 
     # e2e through the public entry point with host buffers
@@ -328,7 +340,7 @@ def main():
         torch.cuda.synchronize()
         e2e_ms = reduce_max(e0.elapsed_time(e1), dist) / args.steps
         in_bytes = 3 * q.numel() * q.element_size()
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+        e2e = {"value": whole_job_tflops(world, flops, e2e_ms), "unit": "TFLOPS", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * out.element_size()}
         del dq, dk, dv
 
