@@ -29,6 +29,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -177,7 +179,7 @@ __device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, i
   }
 }
 
-template <int D, int DT, bool PNQ>
+template <int D, int DT, bool PNQ, bool DUMP>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
   using L = Layout<D>;
   constexpr int NV = PNQ ? D + kOnesRows : D;  // N of the PV MMA
@@ -363,17 +365,20 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     const int row = threadIdx.x;  // TMEM lane and query row within the tile
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     const float c = a.scale_log2;
-    const bool dumping = a.dump != nullptr && bh == a.dump_bh && qt == a.dump_qt;
+    const bool dumping = DUMP && bh == a.dump_bh && qt == a.dump_qt;
     const DumpLayout dl(D, T64);
     float sm = -INFINITY;  // running max of S used for the exponent (raw MMA units)
     float m2 = -INFINITY;  // the same in log2 units, fl32(sm * c)
     float l = 0.f;         // direct placement only (PNQ keeps l in O~ column D)
     bool ok = true;
     bool s_ready = false;  // S(j) was seen complete by the early test during tile j-1
-    for (int j = 0; j < T64; j++) {
+    // one key tile; FULL: all 64 keys are inside N (every tile but possibly the last), so the
+    // main loop carries no masking
+    auto tile = [&](int j, auto full_tag) -> bool {
+      constexpr bool FULL = decltype(full_tag)::value;
       if (!__all_sync(0xFFFFFFFFu, s_ready)) {
         ok = mbar_wait(bar(L::B_S_FULL), j & 1, abort_flag, a.wait_budget);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, ok)) return false;
       }
       tc_fence_after();
       uint32_t s0[32], s1[32];
@@ -393,10 +398,9 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
       }
 
-      const int valid = min(kBN, a.N - j * kBN);
-      const bool full = valid == kBN;  // uniform across the CTA
+      const int valid = FULL ? kBN : a.N - j * kBN;
       float gmax[2];
-      if (full) {
+      if (FULL) {
         gmax[0] = group_max<false>(s0, 0, valid);
         gmax[1] = group_max<false>(s1, 32, valid);
       } else {
@@ -424,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       for (int g = 0; g < 2; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);
       uint32_t w[8];
       float psum[2] = {0.f, 0.f};
-      if (full) {
+      if (FULL) {
         group_codes<false, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
         group_codes<false, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
       } else {
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       // most one phase behind or ahead of the phase waited for here.
       if (any_move) {
         ok = mbar_wait(bar(L::B_O_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, a.wait_budget);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        if (!__all_sync(0xFFFFFFFFu, ok)) return false;
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; cc++) {
@@ -485,7 +489,11 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         dsf[0] = (uint8_t)eb[0];
         dsf[1] = (uint8_t)eb[1];
       }
-    }
+      return true;
+    };
+    const int full_tiles = (a.N % kBN == 0) ? T64 : T64 - 1;
+    for (int j = 0; ok && j < full_tiles; j++) ok = tile(j, std::true_type{});
+    if (ok && full_tiles < T64) ok = tile(T64 - 1, std::false_type{});
     if (ok && T64 >= 2) {  // the last two PV MMAs, one on each O_DONE barrier
       ok = mbar_wait(bar(L::B_O_DONE + (T64 & 1)), ((T64 - 2) >> 1) & 1, abort_flag, a.wait_budget);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -560,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
 template <int D, int DT, bool PNQ>
 static cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
   using L = Layout<D>;
-  auto kern = mxattn_fwd_kernel<D, DT, PNQ>;
+  // the diagnostic dump is a separate instantiation, so the timed kernel carries none of it
+  auto kern = a.dump != nullptr ? mxattn_fwd_kernel<D, DT, PNQ, true> : mxattn_fwd_kernel<D, DT, PNQ, false>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_SMEM);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((a.N + kBM - 1) / kBM), (unsigned)a.BH);
