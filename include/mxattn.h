@@ -112,10 +112,17 @@ typedef struct mxattn_opts {
                            /* tau (log2 units); 0 = eager FlashAttention-2 update       */
   void* workspace;         /* device buffer, see mxattn_workspace_bytes                  */
   size_t workspace_bytes;  /* its size in bytes                                          */
+  long long wait_budget_cycles; /* SM clock cycles a pipeline wait inside the attention     */
+                           /* kernel may last before the kernel gives up and records     */
+                           /* MXATTN_ERR_TIMEOUT; 0 = default (2e9, about one second).  */
+                           /* A test sets it tiny to exercise the expiry path (a wait    */
+                           /* is checked against it only after a first hardware try_wait */
+                           /* returned without the phase); draining in-flight copies and */
+                           /* MMAs always gets the default budget.                       */
 } mxattn_opts;
 
 /* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
- * key_tile 64, rescale_tau 8, no workspace. */
+ * key_tile 64, rescale_tau 8, no workspace, default wait budget. */
 MXATTN_API void mxattn_opts_default(mxattn_opts* opts);
 
 /* Bytes of workspace mxattn_forward needs for this problem (status block plus

@@ -39,7 +39,7 @@ class COpts(ctypes.Structure):
     _fields_ = [("scale_rule", ctypes.c_int), ("qmax", ctypes.c_float), ("pnq", ctypes.c_int),
                 ("rotate", ctypes.c_int), ("dtype", ctypes.c_int), ("key_tile", ctypes.c_int),
                 ("rescale_tau", ctypes.c_float), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("wait_budget_cycles", ctypes.c_longlong)]
 
 
 @dataclass
@@ -50,6 +50,7 @@ class Opts:
     rotate: bool = True
     key_tile: int = 64
     rescale_tau: float = 8.0
+    wait_budget_cycles: int = 0  # 0: the library's default (about one second)
 
 
 def lib_path() -> str:
@@ -124,6 +125,7 @@ def _copts(o: Opts | None, dtype: int, workspace=None) -> COpts:
     load().mxattn_opts_default(ctypes.byref(c))
     c.scale_rule, c.qmax, c.pnq, c.rotate = int(o.scale_rule), float(o.qmax), int(bool(o.pnq)), int(bool(o.rotate))
     c.dtype, c.key_tile, c.rescale_tau = dtype, int(o.key_tile), float(o.rescale_tau)
+    c.wait_budget_cycles = int(o.wait_budget_cycles)
     if workspace is not None:
         c.workspace = ctypes.c_void_p(workspace.data_ptr())
         c.workspace_bytes = workspace.numel() * workspace.element_size()

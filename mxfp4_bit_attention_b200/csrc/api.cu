@@ -60,6 +60,7 @@ mxattn_status check_opts(const mxattn_opts* o) {
   if (o->rotate != 0 && o->rotate != 1) return MXATTN_ERR_INVALID_ARG;
   if (!(o->rescale_tau >= 0.f && std::isfinite(o->rescale_tau))) return MXATTN_ERR_INVALID_ARG;
   if (o->key_tile != 64) return o->key_tile == 128 ? MXATTN_ERR_UNSUPPORTED : MXATTN_ERR_INVALID_ARG;
+  if (o->wait_budget_cycles < 0) return MXATTN_ERR_INVALID_ARG;
   return MXATTN_OK;
 }
 
@@ -105,6 +106,7 @@ void mxattn_opts_default(mxattn_opts* o) {
   o->rescale_tau = 8.0f;
   o->workspace = nullptr;
   o->workspace_bytes = 0;
+  o->wait_budget_cycles = 0;
 }
 
 size_t mxattn_qk_codes_bytes(int B, int H, int N, int d) {
@@ -227,7 +229,7 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
-  a.wait_budget = kWaitBudgetCycles;
+  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.dump = nullptr;
   a.dump_bh = a.dump_qt = -1;
   return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
@@ -265,7 +267,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
-  a.wait_budget = kWaitBudgetCycles;
+  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.dump = dump;
   a.dump_bh = dump_bh;
   a.dump_qt = dump_qt;

@@ -61,6 +61,9 @@ static_assert(kProducerWarp >= 4 && kQkWarp >= 4 && kPvWarp >= 4 && kProducerWar
                   kProducerWarp != kPvWarp && kQkWarp != kPvWarp, "warp roles");
 constexpr int kOnesRows = 16;   // rows appended to V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 256;
+// Budget of the waits that drain in-flight copies and MMAs before a CTA exits (normal or
+// aborted): they always complete, so they get the full default budget whatever the caller set.
+constexpr long long kDrainBudgetCycles = 2000000000LL;
 #ifndef MXATTN_POLY_WORDS
 #define MXATTN_POLY_WORDS 1
 #endif
@@ -260,13 +263,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         bulk_g2s(sb + L::SF_V + s * 512, a.v_scales + t128 * 512, 512, fb);
         issued = j + 1;
       }
-      if (!ok) {
-        raise_abort(abort_flag, a.status, 1);
-        // let every copy already issued land before the CTA can exit
-        mbar_wait(bar(L::B_Q), 0, no_abort, a.wait_budget);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; j++)
-          mbar_wait(bar(L::B_KV_FULL + j % kStages), (j / kStages) & 1, no_abort, a.wait_budget);
-      }
+      if (!ok) raise_abort(abort_flag, a.status, 1);
+      // Let every copy issued land before the CTA can exit, whichever warp gave up (another warp
+      // may abort after this loop finished).  In a normal run these phases have long completed
+      // and nothing newer was issued, so each wait returns at once.
+      mbar_wait(bar(L::B_Q), 0, no_abort, kDrainBudgetCycles);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; j++)
+        mbar_wait(bar(L::B_KV_FULL + j % kStages), (j / kStages) & 1, no_abort, kDrainBudgetCycles);
     }
   } else if (warp == kQkWarp) {
     // ------------------------------------------------------------------ QK issuer
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     // wait for every tcgen05 operation of both issuers before TMEM is released
     if (leader) mma_commit(bar(L::B_DRAIN));
     __syncwarp();
-    mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
+    mbar_wait(bar(L::B_DRAIN), 0, no_abort, kDrainBudgetCycles);
   } else if (warp == kPvWarp) {
     // ------------------------------------------------------------------ PV issuer (same scheme)
     const bool leader = lane == 0;
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     if (!ok && leader) raise_abort(abort_flag, a.status, 4);
     if (leader) mma_commit(bar(L::B_DRAIN));
     __syncwarp();
-    mbar_wait(bar(L::B_DRAIN), 0, no_abort, a.wait_budget);
+    mbar_wait(bar(L::B_DRAIN), 0, no_abort, kDrainBudgetCycles);
   } else if (warp < 4) {
     // ------------------------------------------------------------------ softmax (warps 0-3)
     const int row = threadIdx.x;  // TMEM lane and query row within the tile

@@ -35,6 +35,7 @@ def test_host_only_calls(lib):
     lib.mxattn_opts_default(ctypes.byref(o))
     assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 64)
     assert abs(o.qmax - 7.25) < 1e-7 and abs(o.rescale_tau - 8.0) < 1e-7
+    assert o.wait_budget_cycles == 0  # the library's default budget
     assert lib.mxattn_qk_codes_bytes(1, 2, 200, 128) == 2 * 2 * 128 * 64
     assert lib.mxattn_qk_scales_bytes(1, 2, 200, 128) == 2 * 2 * 512
     assert lib.mxattn_v_codes_bytes(1, 2, 200, 128) == 2 * 4 * 128 * 32
@@ -58,6 +59,9 @@ def test_validation_rejects_before_enqueue(lib):
     o.key_tile = 128
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
     o.key_tile = 64
+    o.wait_budget_cycles = -5
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
+    o.wait_budget_cycles = 0
     o.scale_rule = 3
     o.qmax = 9.0
     assert lib.mxattn_quant_v(fake, 1, 1, 256, 64, P, fake, fake, None) == 1
