@@ -42,19 +42,21 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid,
 
 // ------------------------------------------------------------------------------------------------
 // Q/K: Hadamard rotation + quantization along d into the packed QK operand layout.
-// D/8 threads per token row, 8 consecutive elements per thread; groups of 32 = 4 threads.
+// One thread per MX group (32 consecutive elements of a row, four 16-byte loads in flight), D/32
+// threads per row: butterfly stages h = 1..16 run inside the thread, h = 32 and 64 across the
+// row's threads by shuffles, in the order h = 1, 2, ..., D/2; the group max is the thread's own.
 // Grid: x over (B*H*T128*128) padded token rows, y = 0 for Q, 1 for K.
 // ------------------------------------------------------------------------------------------------
 template <int D, int DT>
 __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
-  constexpr int TPR = D / 8;                 // threads per row
+  constexpr int TPR = D / 32;                // threads per row = groups per row
   constexpr int ROWS = 256 / TPR;            // rows per block
   const int t = threadIdx.x;
-  const int tl = t % TPR;                    // thread within the row
+  const int g = t % TPR;                     // group (and 16-byte code chunk) within the row
   const int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;   // padded row id
   const int64_t T128 = (a.N + 127) / 128;
   const int64_t total = (int64_t)a.BH * T128 * 128;
-  const bool row_ok = prow < total;          // whole warps share this (ROWS multiple of 2)
+  const bool row_ok = prow < total;          // a row's threads are adjacent lanes of one warp
   const int64_t bh = prow / (T128 * 128);
   const int tok = (int)(prow % (T128 * 128));
   const bool valid = row_ok && tok < a.N;
@@ -63,59 +65,75 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
   uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
   uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
 
-  float v[8];
-  load8<DT>(src, ((int64_t)bh * a.N + (valid ? tok : 0)) * D + tl * 8, valid, v);
+  float v[32];
+  const int64_t base = ((int64_t)bh * a.N + (valid ? tok : 0)) * D + g * 32;
+#pragma unroll
+  for (int c = 0; c < 4; c++) load8<DT>(src, base + c * 8, valid, *reinterpret_cast<float(*)[8]>(v + 8 * c));
 
   if (a.rotate) {
-    // stages h = 1, 2, 4 inside the thread
+    // Butterflies (x, y) -> (x + y, x - y), each result rounded once: x - y as fma(y, -1, x).
+    // From h = 2 on, neighbours i, i+1 pair up into f32x2 operations with the same roundings.
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
+    for (int i = 0; i < 32; i += 2) {
+      const float x = v[i], y = v[i + 1];
+      v[i] = __fadd_rn(x, y);
+      v[i + 1] = __fsub_rn(x, y);
+    }
+    const float2 minus1 = make_float2(-1.f, -1.f);
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
+    for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
         if ((i & h) == 0) {
-          const float x = v[i], y = v[i + h];
-          v[i] = __fadd_rn(x, y);
-          v[i + h] = __fsub_rn(x, y);
+          const float2 x = make_float2(v[i], v[i + 1]), y = make_float2(v[i + h], v[i + h + 1]);
+          const float2 sum = __fadd2_rn(x, y), dif = __ffma2_rn(y, minus1, x);
+          v[i] = sum.x; v[i + 1] = sum.y;
+          v[i + h] = dif.x; v[i + h + 1] = dif.y;
         }
       }
     }
-    // stages h = 8 .. D/2 across the TPR lanes of the row (lane bit = h / 8)
+    // stages h = 32 .. D/2 across the TPR lanes of the row (lane bit = h / 32): the lower lane
+    // keeps x + y, the upper one y' = x - y, both as fma(own, +-1, other)
 #pragma unroll
     for (int hb = 1; hb < TPR; hb <<= 1) {
-      const bool upper = (tl & hb) != 0;
+      const float sg = (g & hb) != 0 ? -1.f : 1.f;
+      const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const float other = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
-        v[i] = upper ? __fsub_rn(other, v[i]) : __fadd_rn(v[i], other);
+      for (int i = 0; i < 32; i += 2) {
+        const float o0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
+        const float o1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], hb);
+        const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), sg2, make_float2(o0, o1));
+        v[i] = r.x; v[i + 1] = r.y;
       }
     }
+    const float2 hs = make_float2(a.hadamard_scale, a.hadamard_scale);
 #pragma unroll
-    for (int i = 0; i < 8; i++) v[i] = __fmul_rn(v[i], a.hadamard_scale);
+    for (int i = 0; i < 32; i += 2) {
+      const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), hs);
+      v[i] = r.x; v[i + 1] = r.y;
+    }
   }
 
-  // group amax over the 4 threads of a 32-element group
   float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; i++) amax = fmaxf(amax, fabsf(v[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
   const int e = shared_exponent(amax, a.rule);
   const float inv = pow2_neg(e);
-  const uint32_t w = cvt_e2m1x8(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
-                                __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
-                                __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; q++)
+    w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
+                      __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
+                      __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
   if (!row_ok) return;
   const int r = tok % 128;
   const int64_t tile = bh * T128 + tok / 128;
-  const int c = tl / 4;                                   // group / 16-byte chunk
   const int s = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
   uint8_t* rowp = codes + (tile * 128 + r) * (D / 2);
-  *reinterpret_cast<uint32_t*>(rowp + ((c ^ s) * 16) + (tl % 4) * 4) = w;
-  if ((tl & 3) == 0) {
-    uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
-    atom[c] = (uint8_t)(e + 127);
-    if (D == 64) atom[c + 2] = 0;                         // unused scale slots
-  }
+  *reinterpret_cast<uint4*>(rowp + ((g ^ s) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+  uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
+  atom[g] = (uint8_t)(e + 127);
+  if (D == 64) atom[g + 2] = 0;                           // unused scale slots
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -133,6 +151,8 @@ __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
   const int t = threadIdx.x;
   // stage: 64 tokens x D values, 8 values per thread-iteration
   constexpr int VEC_PER_ROW = D / 8;
+  // a fixed trip count (64 * D / 8 / 256): unrolled, so every thread has all its loads in flight
+#pragma unroll
   for (int idx = t; idx < 64 * VEC_PER_ROW; idx += 256) {
     const int row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
     const int tok = j * 64 + row;
@@ -219,7 +239,7 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
 // ------------------------------------------------------------------------------------------------
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
   const int64_t rows = (int64_t)a.BH * ((a.N + 127) / 128) * 128;
-  const int rows_per_block = 256 / (D / 8);
+  const int rows_per_block = 256 / (D / 32);
   dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
   if (D == 128 && dtype == kBF16) rotate_quant_qk_kernel<128, kBF16><<<grid, 256, 0, s>>>(a);
   else if (D == 128) rotate_quant_qk_kernel<128, kFP32><<<grid, 256, 0, s>>>(a);
