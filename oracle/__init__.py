@@ -75,6 +75,8 @@ def lib():
             L.mxref_attention_rows.argtypes = [P, i64, P, P, i32, i32, f32, ctypes.POINTER(AttnCfg),
                                                P, P, P, P, P, P, P]
             L.mxref_attention_rows.restype = None
+            L.mxref_qmax_sweep.argtypes = [P, i64, i64, i32, P, i32, P, P]
+            L.mxref_qmax_sweep.restype = None
             L.mxref_num_threads.argtypes = []
             L.mxref_num_threads.restype = i32
             _lib = L
@@ -236,6 +238,29 @@ def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=
         res["wsum"] = np.stack(ws)
         res["ocheck"] = np.stack(ocs)
     return res
+
+
+# ----------------------------------------------------------------------------------------------
+# Scale-rule diagnostic: per-block Qmax sweep
+# ----------------------------------------------------------------------------------------------
+
+def qmax_grid(lo: float = 6.0, hi: float = 8.0, step: float = 0.05) -> np.ndarray:
+    """The swept boundaries as fp32 values: lo, lo + step, ..., hi (rounded to fp32 once)."""
+    n = int(round((hi - lo) / step)) + 1
+    return np.array([lo + k * step for k in range(n)], dtype=np.float32)
+
+
+def qmax_sweep(x: np.ndarray, qs: np.ndarray, rotate: bool = False):
+    """Per-block Qmax sweep of the rows of x [rows, cols] (groups of 32 along each row; rows
+    Hadamard-rotated first when rotate).  Returns (counts [nq] uint64: groups for which each q is
+    SSE-optimal, sse_sums [nq] fp64: summed squared error at each q)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    qs = np.ascontiguousarray(qs, dtype=np.float32)
+    rows, cols = x.shape
+    counts = np.zeros(qs.size, np.uint64)
+    sums = np.zeros(qs.size, np.float64)
+    lib().mxref_qmax_sweep(_ptr(x), rows, cols, int(bool(rotate)), _ptr(qs), qs.size, _ptr(counts), _ptr(sums))
+    return counts, sums
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:

@@ -355,6 +355,79 @@ void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const
   }
 }
 
+/*
+ * Per-block Qmax sweep (scale-rule diagnostic; the pages' per-block MSE-optimal boundary study of
+ * Table 4, Pith review page, and the 7.25 argument of Fig. 2 / Theorem 1, applied to synthetic
+ * tensors).
+ *
+ *  x      [rows][cols] fp32, groups of 32 consecutive elements along each row from index 0, the
+ *         tail of the last group zero-padded; rotate: each row (cols = d) is Hadamard-rotated first
+ *         exactly as the Q/K quantizer does.
+ *  qs     nq boundaries q_k (fp32 values, each in [4, 8]).
+ * For each group and each q_k: e_k = the ceiling-rule exponent with boundary q_k (smallest e with
+ * amax <= q_k 2^e, clamped as everywhere); SSE_k = sum_i (x_i - xhat_i)^2 with
+ * xhat_i = E2M1(x_i 2^-e_k) 2^e_k, each difference and square rounded in fp64 and the sum taken in
+ * index order.  counts[k] += 1 for every k whose SSE_k equals the group's smallest (a group counts
+ * for every optimal boundary); sse_sums[k] += SSE_k.  Both outputs are accumulated (the caller
+ * zeroes them); the group count is rows * ceil(cols / 32).
+ */
+void mxref_qmax_sweep(const float* x, int64_t rows, int64_t cols, int rotate, const float* qs, int nq,
+                      uint64_t* counts, double* sse_sums) {
+  const int64_t ng = (cols + 31) / 32;
+  const int nt = omp_get_max_threads();
+  double* part = (double*)calloc((size_t)nt * (size_t)nq, sizeof(double));  /* per-thread sums */
+#pragma omp parallel num_threads(nt)
+  {
+    uint64_t* my_counts = (uint64_t*)calloc((size_t)nq, sizeof(uint64_t));
+    double* my_sums = part + (size_t)omp_get_thread_num() * (size_t)nq;
+    double* sse = (double*)malloc(sizeof(double) * (size_t)nq);
+    float* row = (float*)malloc(sizeof(float) * (size_t)(ng * 32));
+    uint8_t code;
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+      for (int64_t c = 0; c < ng * 32; c++) row[c] = c < cols ? x[r * cols + c] : 0.0f;
+      if (rotate) mxref_fwht_row(row, (int)cols);
+      for (int64_t g = 0; g < ng; g++) {
+        const float* b = row + g * 32;
+        double amax = 0.0;
+        for (int i = 0; i < 32; i++)
+          if (fabs((double)b[i]) > amax) amax = fabs((double)b[i]);
+        double best = INFINITY;
+        int prev_e = 1000;
+        double prev_sse = 0.0;
+        for (int k = 0; k < nq; k++) {
+          const int e = mxref_scale_exponent(amax, MXREF_RULE_CUSTOM, (double)qs[k]);
+          if (e != prev_e) {
+            double s = 0.0;
+            for (int i = 0; i < 32; i++) {
+              code = (uint8_t)mxref_e2m1_encode(ldexp((double)b[i], -e));
+              const double d = (double)b[i] - ldexp(mxref_e2m1_decode(code), e);
+              s += d * d;
+            }
+            prev_e = e;
+            prev_sse = s;
+          }
+          sse[k] = prev_sse;
+          if (prev_sse < best) best = prev_sse;
+        }
+        for (int k = 0; k < nq; k++) {
+          my_sums[k] += sse[k];
+          if (sse[k] == best) my_counts[k]++;
+        }
+      }
+    }
+#pragma omp critical
+    for (int k = 0; k < nq; k++) counts[k] += my_counts[k];
+    free(my_counts);
+    free(sse);
+    free(row);
+  }
+  /* the partial sums are added in thread order, so the result does not depend on timing */
+  for (int t = 0; t < nt; t++)
+    for (int k = 0; k < nq; k++) sse_sums[k] += part[(size_t)t * (size_t)nq + k];
+  free(part);
+}
+
 /* Number of OpenMP threads the oracle runs with. */
 int mxref_num_threads(void) {
   int n = 1;
