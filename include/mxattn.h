@@ -189,6 +189,33 @@ MXATTN_API mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const ui
                                      void* out, void* stream);
 
 /*
+ * Scale-rule diagnostic: per-block Qmax sweep (the per-block MSE-optimal
+ * boundary study of the Pith review page, Table 4, and the 7.25 argument of its
+ * Fig. 2 / Theorem 1, on any tensor).
+ *   x        device, [rows][cols] of `dtype` (MXATTN_BF16 / MXATTN_FP32),
+ *            row-major; groups of 32 consecutive elements along each row from
+ *            index 0, the tail zero-padded.  rotate = 1 Hadamard-rotates every
+ *            row first exactly as mxattn_hadamard_quant_qk does (cols = 64 or
+ *            128).  For V or P~ pass the key-major (transposed) matrix.
+ *   qs       HOST array of nq boundaries (1 <= nq <= 64), each in [4, 8], in
+ *            increasing order; each is a ceiling rule (smallest e with
+ *            amax <= q 2^e).
+ *   counts   device [nq] unsigned 64-bit: += the number of groups for which
+ *            q_k gives the smallest squared reconstruction error (a group counts
+ *            for every optimal q_k: ties are common, the error depends on q only
+ *            through the exponent).
+ *   sse_sums device [nq] fp64: += the summed squared error at q_k (each group's
+ *            error in fp64 in index order; the sum over groups is atomic, so its
+ *            last bits depend on timing).
+ * Both outputs accumulate; the caller zeroes them.  Invalid arguments return
+ * MXATTN_ERR_INVALID_ARG before anything is enqueued.  No counterpart on the
+ * pages beyond the study it reproduces.
+ */
+MXATTN_API mxattn_status mxattn_qmax_sweep(const void* x, int64_t rows, int64_t cols, int dtype, int rotate,
+                                           const float* qs, int nq, unsigned long long* counts,
+                                           double* sse_sums, void* stream);
+
+/*
  * Diagnostic variant of mxattn_attention_mxfp4: identical results, and the CTA
  * that owns query tile dump_qt (128 rows) of head dump_bh (index into B*H)
  * also writes its internal state to `dump` (device buffer of
@@ -200,8 +227,14 @@ MXATTN_API mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const ui
  *   O~ accumulator               fp32 [128][d] before the division by l
  *   l, m                         fp32 [128] each; m = running max of
  *                                S * softmax_scale * log2(e) used for P~
+ *   P~ of every key tile         fp32 [ceil(N/64)][128][64]: the unquantized
+ *                                2^(S * softmax_scale * log2(e) - m) with that
+ *                                tile's running max (0 for keys past N)
+ *   m of every key tile          fp32 [ceil(N/64)][128], after its update
  * (the O~, l, m block starts at the next 16-byte boundary).  Used to measure
- * how many P^ codes differ from the oracle's; the paper has no counterpart.
+ * how many P^ codes differ from the oracle's and to study P~'s quantization
+ * (per-block Qmax sweep, row-sum error decomposition); the paper has no
+ * counterpart.
  */
 MXATTN_API size_t mxattn_attention_dump_bytes(int N, int d);
 MXATTN_API mxattn_status mxattn_attention_mxfp4_dump(

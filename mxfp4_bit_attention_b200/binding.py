@@ -25,7 +25,7 @@ EXPORTS = (
     "mxattn_workspace_init", "mxattn_quantize_mxfp4", "mxattn_hadamard_quant_qk",
     "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
-    "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc",
+    "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
 )
 
 
@@ -90,6 +90,7 @@ def load():
         "mxattn_attention_dump_bytes": ([i32, i32], sz),
         "mxattn_attention_mxfp4_dump": ([P, P, P, P, P, P, i32, i32, i32, i32, f32, PO, P, i32, i32, P, P], i32),
         "mxattn_forward_noalloc": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_qmax_sweep": ([P, i64, i64, i32, i32, P, i32, P, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -216,7 +217,10 @@ def dump_layout(N: int, d: int) -> dict:
     o = (p_scales + T64 * 128 * 2 + 15) // 16 * 16
     l = o + 128 * d * 4
     m = l + 128 * 4
-    return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "total": m + 128 * 4}
+    p_tilde = m + 128 * 4
+    m_tiles = p_tilde + T64 * 128 * 64 * 4
+    return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "p_tilde": p_tilde,
+            "m_tiles": m_tiles, "total": m_tiles + T64 * 128 * 4}
 
 
 def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, dump_qt=0, opts=None,
@@ -246,7 +250,9 @@ def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, 
             "p_scales": raw[L["p_scales"]:L["p_scales"] + T64 * 256].reshape(T64, 128, 2),
             "o": raw[L["o"]:L["l"]].view(np.float32).reshape(128, d),
             "l": raw[L["l"]:L["m"]].view(np.float32).copy(),
-            "m": raw[L["m"]:L["m"] + 512].view(np.float32).copy()}
+            "m": raw[L["m"]:L["m"] + 512].view(np.float32).copy(),
+            "p_tilde": raw[L["p_tilde"]:L["m_tiles"]].view(np.float32).reshape(T64, 128, 64),
+            "m_tiles": raw[L["m_tiles"]:L["total"]].view(np.float32).reshape(T64, 128).copy()}
 
 
 def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None, stream=None):
@@ -278,6 +284,25 @@ def mxattn_forward_noalloc(q, k, v, softmax_scale=None, opts: Opts | None = None
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
         _stream(stream)))
     return out
+
+
+def mxattn_qmax_sweep(x, qs, rotate: bool = False, counts=None, sse_sums=None, stream=None):
+    """Per-block Qmax sweep of the rows of x ([rows, cols], bf16 or fp32, on the GPU) over the
+    increasing boundaries qs (host values in [4, 8]): returns (counts, sse_sums), device tensors
+    of len(qs) -- int64 storage of the unsigned counts of groups for which each q is optimal, and
+    the fp64 summed squared errors.  Given tensors are accumulated into."""
+    import numpy as np
+    import torch
+    rows, cols = x.shape
+    q = np.ascontiguousarray(qs, dtype=np.float32)
+    if counts is None:
+        counts = torch.zeros(q.size, dtype=torch.int64, device=x.device)
+    if sse_sums is None:
+        sse_sums = torch.zeros(q.size, dtype=torch.float64, device=x.device)
+    _check("mxattn_qmax_sweep", load().mxattn_qmax_sweep(
+        _ptr(x), rows, cols, _dtype_code(x), int(bool(rotate)), q.ctypes.data_as(ctypes.c_void_p), q.size,
+        _ptr(counts), _ptr(sse_sums), _stream(stream)))
+    return counts, sse_sums
 
 
 def mxattn_get_device_error(workspace, stream=None) -> int:

@@ -295,6 +295,35 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
                                 ws + c.v_scales, B, H, N, d, softmax_scale, o, out, stream);
 }
 
+mxattn_status mxattn_qmax_sweep(const void* x, int64_t rows, int64_t cols, int dtype, int rotate,
+                                const float* qs, int nq, unsigned long long* counts, double* sse_sums,
+                                void* stream) {
+  if (x == nullptr || qs == nullptr || counts == nullptr || sse_sums == nullptr) return MXATTN_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 1 || nq < 1 || nq > kSweepMaxQ) return MXATTN_ERR_INVALID_ARG;
+  if (dtype != MXATTN_BF16 && dtype != MXATTN_FP32) return MXATTN_ERR_INVALID_ARG;
+  if (rotate != 0 && rotate != 1) return MXATTN_ERR_INVALID_ARG;
+  if (rotate && cols != 64 && cols != 128) return MXATTN_ERR_INVALID_ARG;
+  if (rows * ((cols + 31) / 32) > ((int64_t)1 << 38)) return MXATTN_ERR_UNSUPPORTED;
+  SweepArgs a;
+  a.x = x;
+  a.rows = rows;
+  a.cols = cols;
+  a.rotate = rotate;
+  a.hadamard_scale = (float)(1.0 / std::sqrt((double)cols));
+  a.nq = nq;
+  mxattn_opts o;
+  mxattn_opts_default(&o);
+  o.scale_rule = MXATTN_SCALE_CEIL_CUSTOM;
+  for (int k = 0; k < nq; k++) {
+    if (k > 0 && !(qs[k] > qs[k - 1])) return MXATTN_ERR_INVALID_ARG;
+    o.qmax = qs[k];
+    if (!make_rule(&o, &a.rules[k])) return MXATTN_ERR_INVALID_ARG;  // q in [4, 8]
+  }
+  a.counts = counts;
+  a.sse_sums = sse_sums;
+  return launched(launch_qmax_sweep(a, dtype, as_stream(stream)));
+}
+
 mxattn_status mxattn_get_device_error(const mxattn_opts* o, void* stream) {
   if (o == nullptr) return MXATTN_ERR_INVALID_ARG;
   if (check_workspace(o, kStatusBytes) != MXATTN_OK) return MXATTN_ERR_WORKSPACE;

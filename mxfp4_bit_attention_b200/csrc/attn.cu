@@ -491,6 +491,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         uint8_t* dsf = a.dump + dl.p_scales + ((size_t)j * 128 + row) * 2;
         dsf[0] = (uint8_t)eb[0];
         dsf[1] = (uint8_t)eb[1];
+        // the unquantized tile, relative to this tile's running max (dump only)
+        float* dpt = reinterpret_cast<float*>(a.dump + dl.p_tilde) + ((size_t)j * 128 + row) * 64;
+        for (int i = 0; i < 32; i++) {
+          dpt[i] = i < valid ? ex2_approx(__fmaf_rn(__uint_as_float(s0[i]), c, -m2)) : 0.f;
+          dpt[32 + i] = 32 + i < valid ? ex2_approx(__fmaf_rn(__uint_as_float(s1[i]), c, -m2)) : 0.f;
+        }
+        reinterpret_cast<float*>(a.dump + dl.m_tiles)[(size_t)j * 128 + row] = m2;
       }
       return true;
     };

@@ -40,6 +40,19 @@ struct PlainQuantArgs {
   ScaleRule rule;
 };
 
+// Per-block Qmax sweep (scale-rule diagnostic): boundaries q_k as ceiling rules.
+constexpr int kSweepMaxQ = 64;
+struct SweepArgs {
+  const void* x;
+  int64_t rows, cols;
+  int rotate;                       // Hadamard-rotate each row first (cols = 64 or 128)
+  float hadamard_scale;
+  int nq;
+  ScaleRule rules[kSweepMaxQ];
+  unsigned long long* counts;       // [nq], accumulated
+  double* sse_sums;                 // [nq], accumulated
+};
+
 struct AttnArgs {
   const uint8_t* q_codes;
   const uint8_t* q_scales;
@@ -65,8 +78,11 @@ struct AttnArgs {
 //   P scales               [T64][128][2] bytes (E8M0 of key groups 0 and 1 of the tile)
 //   O accumulator          [128][D] fp32, before the division by l
 //   l, m                   [128] fp32 each (m in log2 units: running max of S * scale * log2 e)
+//   P~                     [T64][128][64] fp32: 2^(S * scale * log2 e - m) with the running max m
+//                          of that tile (0 for keys past N), the unquantized exponential tile
+//   m of every tile        [T64][128] fp32, the running max (log2 units) after each tile's update
 struct DumpLayout {
-  size_t s, p_codes, p_scales, o, l, m, total;
+  size_t s, p_codes, p_scales, o, l, m, p_tilde, m_tiles, total;
   __host__ __device__ DumpLayout(int D, int T64) {
     s = 0;
     p_codes = 2 * 128 * 64 * 4;
@@ -74,7 +90,9 @@ struct DumpLayout {
     o = (p_scales + (size_t)T64 * 128 * 2 + 15) / 16 * 16;
     l = o + (size_t)128 * D * 4;
     m = l + 128 * 4;
-    total = m + 128 * 4;
+    p_tilde = m + 128 * 4;
+    m_tiles = p_tilde + (size_t)T64 * 128 * 64 * 4;
+    total = m_tiles + (size_t)T64 * 128 * 4;
   }
 };
 
@@ -84,6 +102,7 @@ enum { kStatusTimeout = 0x54494D45 /* 'TIME' */ };
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_quant_plain(const PlainQuantArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_qmax_sweep(const SweepArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_fp4_mma_probe(int ctas, int iters, int n, int* status, cudaStream_t s);
 

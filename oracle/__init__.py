@@ -263,6 +263,40 @@ def qmax_sweep(x: np.ndarray, qs: np.ndarray, rotate: bool = False):
     return counts, sums
 
 
+def rowsum_decomposition(p_tilde, p_codes, p_scales, m_tiles):
+    """Row-sum error of direct placement, split by what quantization did to each P~ value.
+
+    p_tilde [T, rows, K]  unquantized exponential tiles (each relative to its tile's running max)
+    p_codes [T, rows, K]  their E2M1 codes (one per byte), p_scales [T, rows, K/32] E8M0 bytes
+    m_tiles [T, rows]     the running max of each tile, log2 units
+    Every value is brought to the final running max (weight 2^(m_t - m_final)).  With direct
+    placement the normalized weights of a row sum to sum(P^) / sum(P~) = 1 + sum of the four
+    contributions below, each the summed (P^ - P~) of its class over sum(P~):
+      zeroing       P~ > 0 quantized to 0
+      saturation    P~ above 6 * 2^e, clipped to the largest code
+      down          other values rounded down, up: values rounded up.
+    Under PNQ the row sum is 1 by construction (Proposition 1).  Returns a dict of per-row arrays
+    (zeroing, saturation, down, up, rowsum_direct)."""
+    pt = np.asarray(p_tilde, dtype=np.float64)
+    T, R, K = pt.shape
+    sc = np.repeat(np.asarray(p_scales, dtype=np.int64), 32, axis=2)
+    codes = np.asarray(p_codes, dtype=np.uint8)
+    mag = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    ph = np.where(codes & 8, -1.0, 1.0) * mag[codes & 7] * np.ldexp(1.0, sc - 127)
+    w = np.exp2(np.asarray(m_tiles, dtype=np.float64) - np.asarray(m_tiles, dtype=np.float64)[-1])[:, :, None]
+    d = (ph - pt) * w
+    top = np.ldexp(6.0, sc - 127)
+    zero = (ph == 0) & (pt > 0)
+    sat = ((codes & 7) == 7) & (pt > top)
+    down = (ph < pt) & ~zero & ~sat
+    up = ph > pt
+    total = (pt * w).sum(axis=(0, 2))
+    res = {name: (d * mask).sum(axis=(0, 2)) / total
+           for name, mask in (("zeroing", zero), ("saturation", sat), ("down", down), ("up", up))}
+    res["rowsum_direct"] = (ph * w).sum(axis=(0, 2)) / total
+    return res
+
+
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to fp32 and then to bf16 (round to nearest, ties to
     even), returned as fp64 values; finite inputs only."""

@@ -70,6 +70,13 @@ def test_validation_rejects_before_enqueue(lib):
     o.scale_rule = 0
     assert lib.mxattn_quantize_mxfp4(fake, 10, 10, 2, P, fake, fake, None) == 1
     assert lib.mxattn_fp4_mma_probe(1, 1, 96, None) == 1
+    qs = (ctypes.c_float * 3)(6.0, 7.25, 8.0)
+    assert lib.mxattn_qmax_sweep(fake, 4, 96, 0, 1, qs, 3, fake, fake, None) == 1       # rotate needs d
+    assert lib.mxattn_qmax_sweep(fake, 4, 128, 0, 0, qs, 0, fake, fake, None) == 1      # nq
+    bad = (ctypes.c_float * 2)(7.25, 7.0)
+    assert lib.mxattn_qmax_sweep(fake, 4, 128, 0, 0, bad, 2, fake, fake, None) == 1     # not increasing
+    out = (ctypes.c_float * 2)(6.0, 9.0)
+    assert lib.mxattn_qmax_sweep(fake, 4, 128, 0, 0, out, 2, fake, fake, None) == 1     # q > 8
 
 
 def test_package_import_does_not_need_the_library(monkeypatch):

@@ -84,3 +84,35 @@ def test_rotation_flag_sweeps_the_rotated_rows():
     c1, s1 = oracle.qmax_sweep(x, QS, rotate=True)
     np.testing.assert_array_equal(c0, c1)
     np.testing.assert_array_equal(s0, s1)
+
+
+def test_rowsum_decomposition_hand_example():
+    """One row, one 64-key tile: group 0 holds the row max 1.0 (UOS exponent -2, step 0.25 at the
+    top), group 1 has max 0.9 (exponent -3: 0.9 / 2^-3 = 7.2 saturates to 6)."""
+    pt = np.zeros((1, 1, 64), np.float32)
+    pt[0, 0, :5] = [1.0, 0.1, 0.05, 0.7, 0.6]
+    pt[0, 0, 32:34] = [0.9, 0.3]
+    codes, scales = oracle.quantize(pt.reshape(1, 64), axis=0)
+    # hand quantization: 1.0 -> 1.0, 0.1 -> 0.125 (up), 0.05 -> 0 (zeroing), 0.7 -> 0.75 (up),
+    # 0.6 -> 0.5 (down); 0.9 -> 0.75 (saturation), 0.3 -> 0.25 (down)
+    assert list(scales[0]) == [127 - 2, 127 - 3]
+    r = oracle.rowsum_decomposition(pt, codes.reshape(1, 1, 64), scales.reshape(1, 1, 2), np.zeros((1, 1)))
+    total = 1.0 + 0.1 + 0.05 + 0.7 + 0.6 + 0.9 + 0.3
+    expect = {"zeroing": -0.05, "saturation": -0.15, "down": -0.1 - 0.05, "up": 0.025 + 0.05}
+    for k, v in expect.items():
+        assert abs(r[k][0] - v / total) < 1e-7, (k, r[k][0], v / total)
+    assert abs(r["rowsum_direct"][0] - (1 + sum(expect.values()) / total)) < 1e-7
+
+
+def test_rowsum_decomposition_rescales_earlier_tiles_to_the_final_max():
+    """Two tiles whose running max moved by 1 (log2): the first tile's values count half."""
+    pt = np.zeros((2, 1, 64), np.float32)
+    pt[0, 0, 0] = 1.0          # exact under its own scale
+    pt[1, 0, 0] = 1.0
+    pt[1, 0, 1] = 0.05         # zeroed (its group's step is 0.25)
+    codes, scales = oracle.quantize(pt.reshape(2, 64), axis=0)
+    m = np.array([[0.0], [1.0]])
+    r = oracle.rowsum_decomposition(pt, codes.reshape(2, 1, 64), scales.reshape(2, 1, 2), m)
+    total = 0.5 * 1.0 + 1.0 + 0.05
+    assert abs(r["zeroing"][0] - (-0.05 / total)) < 1e-7
+    assert r["saturation"][0] == 0 and r["up"][0] == 0 and r["down"][0] == 0
