@@ -251,6 +251,22 @@ MXATTN_API mxattn_status mxattn_forward(const void* q, const void* k, const void
                              void* stream);
 
 /*
+ * Cross-attention (queries and keys of different lengths, e.g. video tokens
+ * attending to text tokens): q and out [B][H][Nq][d], k and v [B][H][Nk][d],
+ * all of opts->dtype, device, 16-byte aligned, non-causal; the same
+ * rotation, quantization and PNQ loop as mxattn_forward, with the key tiles and
+ * the ragged last key tile taken from Nk.  The workspace (256-byte aligned)
+ * holds mxattn_workspace_bytes_cross(B, H, Nq, Nk, d, opts) bytes (0 for
+ * invalid sizes); mxattn_forward_cross(.., N, N, ..) computes what
+ * mxattn_forward does.  Errors as for mxattn_forward.  The pages' video models
+ * use text cross-attention beside self-attention; they fix no API for it.
+ */
+MXATTN_API size_t mxattn_workspace_bytes_cross(int B, int H, int Nq, int Nk, int d, const mxattn_opts* opts);
+MXATTN_API mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, int B, int H, int Nq,
+                                              int Nk, int d, float softmax_scale, const mxattn_opts* opts,
+                                              void* out, void* stream);
+
+/*
  * mxattn_forward without a caller-provided workspace, for callers that cannot
  * allocate device memory: a process whose memory manager has already reserved
  * the GPU's memory (a cudaMalloc would fail or fragment its pool), or a plain C

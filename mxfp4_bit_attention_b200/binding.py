@@ -26,6 +26,7 @@ EXPORTS = (
     "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
     "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
+    "mxattn_workspace_bytes_cross", "mxattn_forward_cross",
 )
 
 
@@ -91,6 +92,8 @@ def load():
         "mxattn_attention_mxfp4_dump": ([P, P, P, P, P, P, i32, i32, i32, i32, f32, PO, P, i32, i32, P, P], i32),
         "mxattn_forward_noalloc": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
         "mxattn_qmax_sweep": ([P, i64, i64, i32, i32, P, i32, P, P, P], i32),
+        "mxattn_workspace_bytes_cross": ([i32, i32, i32, i32, i32, PO], sz),
+        "mxattn_forward_cross": ([P, P, P, i32, i32, i32, i32, i32, f32, PO, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -266,6 +269,25 @@ def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=No
     c = _copts(opts, _dtype_code(q), ws)
     _check("mxattn_forward", load().mxattn_forward(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def mxattn_forward_cross(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None,
+                         stream=None):
+    """Cross-attention: q [B, H, Nq, d] attends to k, v [B, H, Nk, d]; out [B, H, Nq, d]."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    out = out if out is not None else torch.empty_like(q)
+    if workspace is None:
+        nbytes = load().mxattn_workspace_bytes_cross(B, H, Nq, Nk, d, ctypes.byref(_copts(opts, _dtype_code(q))))
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=q.device)
+    c = _copts(opts, _dtype_code(q), workspace)
+    _check("mxattn_forward_cross", load().mxattn_forward_cross(
+        _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
         _stream(stream)))
     return out
 

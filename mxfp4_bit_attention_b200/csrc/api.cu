@@ -68,18 +68,21 @@ struct Carve {
   size_t q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, total;
 };
 
-Carve carve(int B, int H, int N, int d) {
+// Workspace carve-up: status block, then the packed Q operands (Nq tokens) and K/V operands (Nk).
+Carve carve(int B, int H, int Nq, int Nk, int d) {
   Carve c;
   size_t off = kStatusBytes;
-  c.q_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, N, d));
-  c.q_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, N, d));
-  c.k_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, N, d));
-  c.k_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, N, d));
-  c.v_codes = off; off = align256(off + mxattn_v_codes_bytes(B, H, N, d));
-  c.v_scales = off; off = align256(off + mxattn_v_scales_bytes(B, H, N, d));
+  c.q_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, Nq, d));
+  c.q_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, Nq, d));
+  c.k_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, Nk, d));
+  c.k_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, Nk, d));
+  c.v_codes = off; off = align256(off + mxattn_v_codes_bytes(B, H, Nk, d));
+  c.v_scales = off; off = align256(off + mxattn_v_scales_bytes(B, H, Nk, d));
   c.total = off;
   return c;
 }
+
+Carve carve(int B, int H, int N, int d) { return carve(B, H, N, N, d); }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -159,11 +162,16 @@ mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, i
   return launched(launch_quant_plain(a, o->dtype, as_stream(stream)));
 }
 
-mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
-                                       const mxattn_opts* o, uint8_t* q_codes, uint8_t* q_scales,
-                                       uint8_t* k_codes, uint8_t* k_scales, void* stream) {
-  if (!sizes_ok(B, H, N, d)) return (B >= 1 && H >= 1 && N >= 1 && (d == 64 || d == 128)) ? MXATTN_ERR_UNSUPPORTED
-                                                                                          : MXATTN_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Q (Nq tokens) and K (Nk tokens) rotated and quantized in one launch.
+mxattn_status quant_qk(const void* q, const void* k, int B, int H, int Nq, int Nk, int d, const mxattn_opts* o,
+                       uint8_t* q_codes, uint8_t* q_scales, uint8_t* k_codes, uint8_t* k_scales, void* stream) {
+  if (!sizes_ok(B, H, Nq, d) || !sizes_ok(B, H, Nk, d))
+    return (B >= 1 && H >= 1 && Nq >= 1 && Nk >= 1 && (d == 64 || d == 128)) ? MXATTN_ERR_UNSUPPORTED
+                                                                               : MXATTN_ERR_INVALID_ARG;
   if (!q || !k || !q_codes || !q_scales || !k_codes || !k_scales) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
@@ -176,11 +184,22 @@ mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int 
   a.k_codes = k_codes;
   a.k_scales = k_scales;
   a.BH = B * H;
-  a.N = N;
+  a.N = Nq;
+  a.Nk = Nk;
   a.rotate = o->rotate;
   a.hadamard_scale = (float)(1.0 / std::sqrt((double)d));
   make_rule(o, &a.rule);
   return launched(launch_rotate_quant_qk(a, d, o->dtype, as_stream(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+mxattn_status mxattn_hadamard_quant_qk(const void* q, const void* k, int B, int H, int N, int d,
+                                       const mxattn_opts* o, uint8_t* q_codes, uint8_t* q_scales,
+                                       uint8_t* k_codes, uint8_t* k_scales, void* stream) {
+  return quant_qk(q, k, B, H, N, N, d, o, q_codes, q_scales, k_codes, k_scales, stream);
 }
 
 mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mxattn_opts* o, uint8_t* v_codes,
@@ -200,11 +219,14 @@ mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mx
   return launched(launch_quant_v(a, d, o->dtype, as_stream(stream)));
 }
 
-mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
-                                     const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales,
-                                     int B, int H, int N, int d, float softmax_scale, const mxattn_opts* o,
-                                     void* out, void* stream) {
-  if (!sizes_ok(B, H, N, d)) return MXATTN_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                        const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales, int B, int H,
+                        int Nq, int Nk, int d, float softmax_scale, const mxattn_opts* o, void* out, void* stream) {
+  if (!sizes_ok(B, H, Nq, d) || !sizes_ok(B, H, Nk, d)) return MXATTN_ERR_INVALID_ARG;
   if (!q_codes || !q_scales || !k_codes || !k_scales || !v_codes || !v_scales || !out) return MXATTN_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
@@ -224,7 +246,8 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
   a.out = out;
   a.status = reinterpret_cast<int*>(o->workspace);
   a.BH = B * H;
-  a.N = N;
+  a.N = Nq;
+  a.Nk = Nk;
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
@@ -233,6 +256,18 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
   a.dump = nullptr;
   a.dump_bh = a.dump_qt = -1;
   return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
+                                     const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales,
+                                     int B, int H, int N, int d, float softmax_scale, const mxattn_opts* o,
+                                     void* out, void* stream) {
+  return attention(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, B, H, N, N, d, softmax_scale, o, out,
+                   stream);
 }
 
 size_t mxattn_attention_dump_bytes(int N, int d) {
@@ -263,6 +298,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   a.status = reinterpret_cast<int*>(o->workspace);
   a.BH = B * H;
   a.N = N;
+  a.Nk = N;
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
@@ -293,6 +329,32 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
   if (st != MXATTN_OK) return st;
   return mxattn_attention_mxfp4(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes,
                                 ws + c.v_scales, B, H, N, d, softmax_scale, o, out, stream);
+}
+
+size_t mxattn_workspace_bytes_cross(int B, int H, int Nq, int Nk, int d, const mxattn_opts* opts) {
+  (void)opts;
+  if (!sizes_ok(B, H, Nq, d) || !sizes_ok(B, H, Nk, d)) return 0;
+  return carve(B, H, Nq, Nk, d).total;
+}
+
+mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, int B, int H, int Nq, int Nk, int d,
+                                   float softmax_scale, const mxattn_opts* o, void* out, void* stream) {
+  if (!sizes_ok(B, H, Nq, d) || !sizes_ok(B, H, Nk, d)) return MXATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  const Carve c = carve(B, H, Nq, Nk, d);
+  st = check_workspace(o, c.total);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
+  st = quant_qk(q, k, B, H, Nq, Nk, d, o, ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, stream);
+  if (st != MXATTN_OK) return st;
+  st = mxattn_quant_v(v, B, H, Nk, d, o, ws + c.v_codes, ws + c.v_scales, stream);
+  if (st != MXATTN_OK) return st;
+  return attention(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes, ws + c.v_scales,
+                   B, H, Nq, Nk, d, softmax_scale, o, out, stream);
 }
 
 mxattn_status mxattn_qmax_sweep(const void* x, int64_t rows, int64_t cols, int dtype, int rotate,

@@ -190,8 +190,9 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T128 = (a.N + 127) / 128;
-  const int T64 = (a.N + 63) / 64;
+  const int T128 = (a.N + 127) / 128;   // query tiles of a head
+  const int T128k = (a.Nk + 127) / 128; // 128-key operand tiles of a head
+  const int T64 = (a.Nk + 63) / 64;     // 64-key tiles swept by the CTA
   const int qt = blockIdx.x;
   const int bh = blockIdx.y;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::ABORT);
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           if (!ok) break;
         }
         const uint32_t fb = bar(L::B_KV_FULL + s);
-        const size_t t128 = (size_t)bh * T128 + j / 2;
+        const size_t t128 = (size_t)bh * T128k + j / 2;
         mbar_arrive_expect_tx(fb, L::K_BYTES + L::V_BYTES + 1024);
         bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES,
                  a.k_codes + (t128 * kBM + (j % 2) * kBN) * (size_t)(D / 2), L::K_BYTES, fb);
@@ -401,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
       }
 
-      const int valid = FULL ? kBN : a.N - j * kBN;
+      const int valid = FULL ? kBN : a.Nk - j * kBN;
       float gmax[2];
       if (FULL) {
         gmax[0] = group_max<false>(s0, 0, valid);
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
       return true;
     };
-    const int full_tiles = (a.N % kBN == 0) ? T64 : T64 - 1;
+    const int full_tiles = (a.Nk % kBN == 0) ? T64 : T64 - 1;
     for (int j = 0; ok && j < full_tiles; j++) ok = tile(j, std::true_type{});
     if (ok && full_tiles < T64) ok = tile(T64 - 1, std::false_type{});
     if (ok && T64 >= 2) {  // the last two PV MMAs, one on each O_DONE barrier

@@ -17,7 +17,8 @@ struct QKQuantArgs {
   uint8_t* q_scales;
   uint8_t* k_codes;
   uint8_t* k_scales;
-  int BH, N;
+  int BH, N;             // N: tokens of Q
+  int Nk;                // tokens of K (= N for self-attention)
   int rotate;
   float hadamard_scale;  // fl32(1/sqrt(d))
   ScaleRule rule;
@@ -62,7 +63,8 @@ struct AttnArgs {
   const uint8_t* v_scales;
   void* out;
   int* status;           // workspace status block (error word at [0], detail at [1..3])
-  int BH, N;
+  int BH, N;             // N: query rows per head
+  int Nk;                // keys (and values) per head (= N for self-attention)
   float scale_log2;      // softmax_scale * log2(e)
   float tau;             // lazy max threshold, log2 units
   int pnq;

@@ -45,7 +45,7 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid,
 // One thread per MX group (32 consecutive elements of a row, four 16-byte loads in flight), D/32
 // threads per row: butterfly stages h = 1..16 run inside the thread, h = 32 and 64 across the
 // row's threads by shuffles, in the order h = 1, 2, ..., D/2; the group max is the thread's own.
-// Grid: x over (B*H*T128*128) padded token rows, y = 0 for Q, 1 for K.
+// Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K.
 // ------------------------------------------------------------------------------------------------
 template <int D, int DT>
 __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
@@ -54,19 +54,20 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
   const int t = threadIdx.x;
   const int g = t % TPR;                     // group (and 16-byte code chunk) within the row
   const int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;   // padded row id
-  const int64_t T128 = (a.N + 127) / 128;
+  const int Nt = blockIdx.y == 0 ? a.N : a.Nk;  // tokens of this tensor
+  const int64_t T128 = (Nt + 127) / 128;
   const int64_t total = (int64_t)a.BH * T128 * 128;
   const bool row_ok = prow < total;          // a row's threads are adjacent lanes of one warp
   const int64_t bh = prow / (T128 * 128);
   const int tok = (int)(prow % (T128 * 128));
-  const bool valid = row_ok && tok < a.N;
+  const bool valid = row_ok && tok < Nt;
 
   const void* src = blockIdx.y == 0 ? a.q : a.k;
   uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
   uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
 
   float v[32];
-  const int64_t base = ((int64_t)bh * a.N + (valid ? tok : 0)) * D + g * 32;
+  const int64_t base = ((int64_t)bh * Nt + (valid ? tok : 0)) * D + g * 32;
 #pragma unroll
   for (int c = 0; c < 4; c++) load8<DT>(src, base + c * 8, valid, *reinterpret_cast<float(*)[8]>(v + 8 * c));
 
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
 // Launchers
 // ------------------------------------------------------------------------------------------------
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
-  const int64_t rows = (int64_t)a.BH * ((a.N + 127) / 128) * 128;
+  const int64_t rows = (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
   const int rows_per_block = 256 / (D / 32);
   dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
   if (D == 128 && dtype == kBF16) rotate_quant_qk_kernel<128, kBF16><<<grid, 256, 0, s>>>(a);

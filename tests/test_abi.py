@@ -42,6 +42,11 @@ def test_host_only_calls(lib):
     assert lib.mxattn_v_scales_bytes(1, 2, 200, 64) == 2 * 2 * 512
     assert lib.mxattn_workspace_bytes(1, 1, 256, 96, ctypes.byref(o)) == 0
     assert lib.mxattn_workspace_bytes(1, 40, 75600, 128, ctypes.byref(o)) > 256
+    assert lib.mxattn_workspace_bytes_cross(2, 3, 500, 500, 128, ctypes.byref(o)) == \
+        lib.mxattn_workspace_bytes(2, 3, 500, 128, ctypes.byref(o))
+    assert lib.mxattn_workspace_bytes_cross(1, 4, 75600, 512, 128, ctypes.byref(o)) < \
+        lib.mxattn_workspace_bytes(1, 4, 75600, 128, ctypes.byref(o))
+    assert lib.mxattn_workspace_bytes_cross(1, 4, 100, 0, 128, ctypes.byref(o)) == 0
     assert lib.mxattn_status_string(5) == b"MXATTN_ERR_TIMEOUT"
 
 
@@ -56,6 +61,9 @@ def test_validation_rejects_before_enqueue(lib):
     assert lib.mxattn_forward(None, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1       # null
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, -1.0, P, fake, None) == 1      # scale
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3       # no workspace
+    assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 0, 64, 0.1, P, fake, None) == 1    # Nk
+    assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 96, 0.1, P, fake, None) == 1  # d
+    assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 64, 0.1, P, fake, None) == 3  # no workspace
     o.key_tile = 128
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
     o.key_tile = 64

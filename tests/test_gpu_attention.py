@@ -53,6 +53,15 @@ def test_tiny_modes(pnq, rule):
     check(got, ref, f"pnq={pnq} rule={rule}")
 
 
+@pytest.mark.parametrize("q", [7.0, 7.5])  # 7.0: the OAS rule of Appendix G (Eq. 96); 7.5: above UOS
+@pytest.mark.parametrize("pnq", [True, False])
+def test_tiny_custom_boundary(q, pnq):
+    w = inputs.WORKLOADS["tiny"]
+    g = inputs.generate(w)
+    got, ref = run(g, w, binding.Opts(scale_rule=binding.SCALE_CEIL_CUSTOM, qmax=q, pnq=pnq))
+    check(got, ref, f"q={q} pnq={pnq}")
+
+
 @pytest.mark.parametrize("tau", [0.0, 8.0])
 @pytest.mark.parametrize("rotate", [True, False])
 def test_tiny_tau_rotate(tau, rotate):

@@ -8,7 +8,8 @@
    fraction that differ is printed, and bounded well below what the attention
    tolerance could absorb.
 2. Error against exact attention.  For the outlier workload, the MXFP4 output
-   under the UOS (Qmax = 7.25), Qmax = 6 and OCP scale rules, each with PNQ on
+   under the UOS (Qmax = 7.25), Qmax = 6 and OCP scale rules and the ceiling boundaries 7.0 (the
+   OAS rule) and 7.5, each with PNQ on
    and off, is compared with fp32 softmax attention on the unquantized inputs.
    The numbers are printed; the asserts only bound them loosely, since the
    pages fix no ranking for synthetic data.
@@ -83,11 +84,15 @@ def test_error_against_exact_attention_by_scale_rule():
     q, k, v = (to_device(g[n], w.dtype, (1, w.H, w.N, w.d)) for n in "qkv")
     scale = float(np.float32(w.d ** -0.5))
     exact = _exact_attention(q, k, v, scale)
-    modes = [("UOS 7.25", binding.SCALE_UOS), ("Qmax 6", binding.SCALE_QMAX6), ("OCP", binding.SCALE_OCP)]
+    modes = [("UOS 7.25", binding.SCALE_UOS, 7.25), ("Qmax 6", binding.SCALE_QMAX6, 6.0),
+             ("OCP", binding.SCALE_OCP, 7.25),
+             # the boundary ablation: q = 7 is the OAS rule of Appendix G (Eq. 96), 7.5 lies above UOS
+             ("q 7.0 (OAS)", binding.SCALE_CEIL_CUSTOM, 7.0), ("q 7.5", binding.SCALE_CEIL_CUSTOM, 7.5)]
     table = {}
-    for label, rule in modes:
+    for label, rule, qmax in modes:
         for pnq in (True, False):
-            out = binding.mxattn_forward(q, k, v, scale, binding.Opts(scale_rule=rule, pnq=pnq)).float()
+            opts = binding.Opts(scale_rule=rule, qmax=qmax, pnq=pnq)
+            out = binding.mxattn_forward(q, k, v, scale, opts).float()
             err = (out - exact).double()
             rel = float(err.norm() / exact.double().norm())
             table[f"{label}, PNQ {'on' if pnq else 'off'}"] = rel

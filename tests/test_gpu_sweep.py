@@ -23,6 +23,8 @@ pytestmark = pytest.mark.gpu
 
 QS = oracle.qmax_grid()
 I725 = int(np.argmin(np.abs(QS - 7.25)))
+I700 = int(np.argmin(np.abs(QS - 7.0)))
+I750 = int(np.argmin(np.abs(QS - 7.5)))
 
 
 def _sweep_both(x_dev, x_host, rotate, label):
@@ -35,7 +37,9 @@ def _sweep_both(x_dev, x_host, rotate, label):
     groups = x_host.shape[0] * ((x_host.shape[1] + 31) // 32)
     print("DIAG " + json.dumps({"diag": "qmax_sweep", "tensor": label, "groups": groups,
                                 "mode_q": float(QS[int(np.argmax(got_c))]),
+                                "fraction_optimal_at_7.00": float(got_c[I700]) / groups,
                                 "fraction_optimal_at_7.25": float(got_c[I725]) / groups,
+                                "fraction_optimal_at_7.50": float(got_c[I750]) / groups,
                                 "fraction_optimal_at_6.00": float(got_c[0]) / groups,
                                 "fraction_optimal_at_8.00": float(got_c[-1]) / groups,
                                 "argmin_mean_sse_q": float(QS[int(np.argmin(got_s))])}))
