@@ -26,7 +26,8 @@ EXPORTS = (
     "mxattn_quant_v", "mxattn_attention_mxfp4", "mxattn_forward", "mxattn_get_device_error",
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
     "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
-    "mxattn_workspace_bytes_cross", "mxattn_forward_cross",
+    "mxattn_workspace_bytes_cross", "mxattn_forward_cross", "mxattn_workspace_bytes_host",
+    "mxattn_forward_host",
 )
 
 
@@ -94,6 +95,8 @@ def load():
         "mxattn_qmax_sweep": ([P, i64, i64, i32, i32, P, i32, P, P, P], i32),
         "mxattn_workspace_bytes_cross": ([i32, i32, i32, i32, i32, PO], sz),
         "mxattn_forward_cross": ([P, P, P, i32, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_workspace_bytes_host": ([i32, i32, i32, i32, PO], sz),
+        "mxattn_forward_host": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -270,6 +273,26 @@ def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=No
     _check("mxattn_forward", load().mxattn_forward(
         _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
         _stream(stream)))
+    return out
+
+
+def mxattn_forward_host(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None,
+                        stream=None):
+    """The forward pass from host tensors q, k, v [B, H, N, d] (page-locked for the transfers to
+    overlap the kernels) into the host tensor `out`; chunks of heads pipeline their copies with
+    the computation.  Synchronize the stream before reading `out`."""
+    import torch
+    B, H, N, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    out = out if out is not None else torch.empty_like(q).pin_memory()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if workspace is None:
+        nbytes = load().mxattn_workspace_bytes_host(B, H, N, d, ctypes.byref(_copts(opts, _dtype_code(q))))
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    c = _copts(opts, _dtype_code(q), workspace)
+    _check("mxattn_forward_host", load().mxattn_forward_host(
+        _ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(softmax_scale), ctypes.byref(c), _ptr(out), _stream(stream)))
     return out
 
 

@@ -357,6 +357,142 @@ mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, 
                    B, H, Nq, Nk, d, softmax_scale, o, out, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Host-buffer forward: the heads are processed in chunks, each chunk an independent problem.
+#ifndef MXATTN_HOST_CHUNKS
+#define MXATTN_HOST_CHUNKS 40
+#endif
+constexpr int kHostChunks = MXATTN_HOST_CHUNKS;
+
+struct HostPlan {
+  int BH, hc, nch;               // heads, heads per chunk, chunks
+  size_t head_bytes;             // one head of q, k, v or out
+  size_t in_off[2], out_off[2];  // double-buffered q|k|v and out staging
+  size_t qc, qs, kc, ks, vc, vs; // packed operands of one chunk
+  size_t total;
+};
+
+HostPlan host_plan(int B, int H, int N, int d, int dtype) {
+  HostPlan p;
+  p.BH = B * H;
+  int nch = p.BH < kHostChunks ? p.BH : kHostChunks;
+  p.hc = (p.BH + nch - 1) / nch;
+  p.nch = (p.BH + p.hc - 1) / p.hc;
+  p.head_bytes = (size_t)N * d * (dtype == MXATTN_BF16 ? 2 : 4);
+  size_t off = kStatusBytes;
+  for (int b = 0; b < 2; b++) {
+    p.in_off[b] = off;
+    off = align256(off + 3 * (size_t)p.hc * p.head_bytes);
+  }
+  for (int b = 0; b < 2; b++) {
+    p.out_off[b] = off;
+    off = align256(off + (size_t)p.hc * p.head_bytes);
+  }
+  p.qc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
+  p.qs = off; off = align256(off + mxattn_qk_scales_bytes(1, p.hc, N, d));
+  p.kc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
+  p.ks = off; off = align256(off + mxattn_qk_scales_bytes(1, p.hc, N, d));
+  p.vc = off; off = align256(off + mxattn_v_codes_bytes(1, p.hc, N, d));
+  p.vs = off; off = align256(off + mxattn_v_scales_bytes(1, p.hc, N, d));
+  p.total = off;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mxattn_workspace_bytes_host(int B, int H, int N, int d, const mxattn_opts* opts) {
+  if (!sizes_ok(B, H, N, d)) return 0;
+  return host_plan(B, H, N, d, opts != nullptr ? opts->dtype : MXATTN_BF16).total;
+}
+
+mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const void* v_host, int B, int H, int N,
+                                  int d, float softmax_scale, const mxattn_opts* o, void* out_host, void* stream) {
+  if (!sizes_ok(B, H, N, d)) return MXATTN_ERR_INVALID_ARG;
+  if (!q_host || !k_host || !v_host || !out_host) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  const HostPlan p = host_plan(B, H, N, d, o->dtype);
+  st = check_workspace(o, p.total);
+  if (st != MXATTN_OK) return st;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
+  const uint8_t* qh = reinterpret_cast<const uint8_t*>(q_host);
+  const uint8_t* kh = reinterpret_cast<const uint8_t*>(k_host);
+  const uint8_t* vh = reinterpret_cast<const uint8_t*>(v_host);
+  uint8_t* oh = reinterpret_cast<uint8_t*>(out_host);
+  cudaStream_t s = as_stream(stream);
+
+  // copies in on s_in, compute on the caller's stream, copies out on s_out; every cross-stream
+  // order is an event, and the caller's stream finally waits for the last copies out
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess;
+  for (int b = 0; ok && b < 2; b++)
+    ok = cudaEventCreateWithFlags(&ev_in[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_comp[b], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_out[b], cudaEventDisableTiming) == cudaSuccess;
+  // work already on the caller's stream comes first
+  ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+  st = ok ? MXATTN_OK : MXATTN_ERR_CUDA;
+  for (int c = 0; st == MXATTN_OK && c < p.nch; c++) {
+    const int b = c & 1;
+    const int h0 = c * p.hc;
+    const int hn = p.BH - h0 < p.hc ? p.BH - h0 : p.hc;
+    const size_t bytes = (size_t)hn * p.head_bytes, src = (size_t)h0 * p.head_bytes;
+    uint8_t* in = ws + p.in_off[b];
+    uint8_t* qd = in;
+    uint8_t* kd = in + (size_t)p.hc * p.head_bytes;
+    uint8_t* vd = in + 2 * (size_t)p.hc * p.head_bytes;
+    uint8_t* od = ws + p.out_off[b];
+    // inputs of chunk c into buffer b once chunk c-2 has finished reading it
+    if (c >= 2 && cudaStreamWaitEvent(s_in, ev_comp[b], 0) != cudaSuccess) { st = MXATTN_ERR_CUDA; break; }
+    if (cudaMemcpyAsync(qd, qh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(kd, kh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(vd, vh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaEventRecord(ev_in[b], s_in) != cudaSuccess || cudaStreamWaitEvent(s, ev_in[b], 0) != cudaSuccess) {
+      st = MXATTN_ERR_CUDA;
+      break;
+    }
+    // the output buffer b is free once chunk c-2's copy out has finished
+    if (c >= 2 && cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess) { st = MXATTN_ERR_CUDA; break; }
+    st = quant_qk(qd, kd, 1, hn, N, N, d, o, ws + p.qc, ws + p.qs, ws + p.kc, ws + p.ks, stream);
+    if (st == MXATTN_OK) st = mxattn_quant_v(vd, 1, hn, N, d, o, ws + p.vc, ws + p.vs, stream);
+    if (st == MXATTN_OK)
+      st = attention(ws + p.qc, ws + p.qs, ws + p.kc, ws + p.ks, ws + p.vc, ws + p.vs, 1, hn, N, N, d, softmax_scale,
+                     o, od, stream);
+    if (st != MXATTN_OK) break;
+    if (cudaEventRecord(ev_comp[b], s) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_comp[b], 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + src, od, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
+        cudaEventRecord(ev_out[b], s_out) != cudaSuccess) {
+      st = MXATTN_ERR_CUDA;
+      break;
+    }
+  }
+  // join: the caller's stream waits for every copy out (and, through them, everything else)
+  for (int b = 0; b < 2 && ev_out[b] != nullptr; b++)
+    if (cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess && st == MXATTN_OK) st = MXATTN_ERR_CUDA;
+  if (ev_start != nullptr && cudaStreamWaitEvent(s, ev_start, 0) != cudaSuccess && st == MXATTN_OK)
+    st = MXATTN_ERR_CUDA;
+  // streams and events are released once their pending work completes
+  for (int b = 0; b < 2; b++) {
+    if (ev_in[b]) cudaEventDestroy(ev_in[b]);
+    if (ev_comp[b]) cudaEventDestroy(ev_comp[b]);
+    if (ev_out[b]) cudaEventDestroy(ev_out[b]);
+  }
+  if (ev_start) cudaEventDestroy(ev_start);
+  if (s_in) cudaStreamDestroy(s_in);
+  if (s_out) cudaStreamDestroy(s_out);
+  return st;
+}
+
 mxattn_status mxattn_qmax_sweep(const void* x, int64_t rows, int64_t cols, int dtype, int rotate,
                                 const float* qs, int nq, unsigned long long* counts, double* sse_sums,
                                 void* stream) {

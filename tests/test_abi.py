@@ -47,6 +47,9 @@ def test_host_only_calls(lib):
     assert lib.mxattn_workspace_bytes_cross(1, 4, 75600, 512, 128, ctypes.byref(o)) < \
         lib.mxattn_workspace_bytes(1, 4, 75600, 128, ctypes.byref(o))
     assert lib.mxattn_workspace_bytes_cross(1, 4, 100, 0, 128, ctypes.byref(o)) == 0
+    # staging for two chunks of 4 heads, far below the 2.3 GB of all 40 heads' bf16 inputs
+    assert 0 < lib.mxattn_workspace_bytes_host(1, 40, 75600, 128, ctypes.byref(o)) < 3 * 40 * 75600 * 128 * 2 // 3
+    assert lib.mxattn_workspace_bytes_host(1, 1, 0, 128, ctypes.byref(o)) == 0
     assert lib.mxattn_status_string(5) == b"MXATTN_ERR_TIMEOUT"
 
 
@@ -64,6 +67,8 @@ def test_validation_rejects_before_enqueue(lib):
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 0, 64, 0.1, P, fake, None) == 1    # Nk
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 96, 0.1, P, fake, None) == 1  # d
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 64, 0.1, P, fake, None) == 3  # no workspace
+    assert lib.mxattn_forward_host(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3       # no workspace
+    assert lib.mxattn_forward_host(None, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1       # null
     o.key_tile = 128
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
     o.key_tile = 64
