@@ -45,7 +45,8 @@ def build(force: bool = False) -> str:
 
 class AttnCfg(ctypes.Structure):
     _fields_ = [("key_tile", ctypes.c_int), ("pnq", ctypes.c_int), ("quant_p", ctypes.c_int),
-                ("rule", ctypes.c_int), ("qmax", ctypes.c_double), ("tau", ctypes.c_double)]
+                ("rule", ctypes.c_int), ("qmax", ctypes.c_double), ("tau", ctypes.c_double),
+                ("qpos", ctypes.c_void_p)]
 
 
 def lib():
@@ -162,17 +163,20 @@ def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------------------------
 
 def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=True, rule=RULE_UOS,
-                   qmax=7.25, tau=0.0, weights=False, codes=False):
+                   qmax=7.25, tau=0.0, weights=False, codes=False, qpos=None):
     """Online-softmax attention with PNQ for query rows qd [n, d] against
     kd, vd [N, d] (fp64 values).  Returns dict(out, m, l[, wsum, ocheck]
-    [, p_codes [n, ntiles*key_tile], p_scales [n, ntiles*key_tile/32]])."""
+    [, p_codes [n, ntiles*key_tile], p_scales [n, ntiles*key_tile/32]]).  qpos: causal masking,
+    row i sees keys 0..qpos[i] (None: all keys)."""
     qd = np.ascontiguousarray(qd, dtype=np.float64)
     kd = np.ascontiguousarray(kd, dtype=np.float64)
     vd = np.ascontiguousarray(vd, dtype=np.float64)
     n, d = qd.shape
     N = kd.shape[0]
     assert kd.shape == (N, d) and vd.shape == (N, d) and key_tile % 32 == 0
-    cfg = AttnCfg(int(key_tile), int(bool(pnq)), int(bool(quant_p)), int(rule), float(qmax), float(tau))
+    qp = None if qpos is None else np.ascontiguousarray(qpos, dtype=np.int64)
+    cfg = AttnCfg(int(key_tile), int(bool(pnq)), int(bool(quant_p)), int(rule), float(qmax), float(tau),
+                  None if qp is None else qp.ctypes.data)
     out = np.empty((n, d), np.float64)
     m = np.empty(n, np.float64)
     l = np.empty(n, np.float64)
@@ -214,11 +218,12 @@ def prepare_head(q, k, v, rotate=True, rule=RULE_UOS, qmax=7.25, quant=True):
 
 
 def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=7.25, pnq=True,
-                 key_tile=64, tau=0.0, quant=True, weights=False):
+                 key_tile=64, tau=0.0, quant=True, weights=False, causal=False):
     """MXAttention forward for selected query rows of every head.
 
     q, k, v: fp32 arrays [BH, N, d] (exact upcasts of the inputs).
     rows:    int array of query indices (same rows for every head).
+    causal:  each row sees only the keys up to its own index (self-attention, top-left aligned).
     Returns dict with out [BH, len(rows), d] (fp64) and m, l [BH, len(rows)].
     """
     BH, N, d = q.shape
@@ -226,7 +231,8 @@ def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=
     outs, ms, ls, ws, ocs = [], [], [], [], []
     for h in range(BH):
         qd, kd, vd = prepare_head(q[h][rows], k[h], v[h], rotate, rule, qmax, quant)
-        r = attention_rows(qd, kd, vd, softmax_scale, key_tile, pnq, quant, rule, qmax, tau, weights)
+        r = attention_rows(qd, kd, vd, softmax_scale, key_tile, pnq, quant, rule, qmax, tau, weights,
+                           qpos=rows if causal else None)
         outs.append(r["out"])
         ms.append(r["m"])
         ls.append(r["l"])

@@ -228,6 +228,8 @@ typedef struct {
   int rule;       /* scale rule for the exponential tile                    */
   double qmax;    /* boundary for MXREF_RULE_CUSTOM                           */
   double tau;     /* lazy max update threshold in log2 units; 0 = eager      */
+  const int64_t* qpos; /* causal masking: key k is seen by row r only if k <= qpos[r]
+                          (the row's position in the sequence); NULL: every key     */
 } mxref_attn_cfg;
 
 /*
@@ -277,12 +279,16 @@ void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const
 #pragma omp for schedule(dynamic, 1)
     for (int64_t r = 0; r < nrows; r++) {
       const double* qr = q + r * d;
+      /* keys this row sees: the first `lim` (all N, or up to its position under causal masking);
+         tiles past them hold only masked keys: no max move, P~ = 0 */
+      const int64_t lim = cfg->qpos ? (cfg->qpos[r] + 1 < N ? cfg->qpos[r] + 1 : N) : N;
       double l = 0.0;
       float m = -INFINITY;
       for (int c = 0; c < d; c++) acc[c] = 0.0;
       for (int t = 0; t < ntiles; t++) {
         int k0 = t * T;
-        int nk = N - k0 < T ? N - k0 : T;
+        int nk = lim - k0 < T ? (int)(lim - k0) : T;
+        if (nk < 0) nk = 0;
         float mt = -INFINITY;
         for (int j = 0; j < nk; j++) {
           const double* kr = k + (int64_t)(k0 + j) * d;
@@ -332,7 +338,8 @@ void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const
           for (int c = 0; c < d; c++) oc[c] = 0.0;
         for (int t = ntiles - 1; t >= 0; t--) {
           int k0 = t * T;
-          int nk = N - k0 < T ? N - k0 : T;
+          int nk = lim - k0 < T ? (int)(lim - k0) : T;
+          if (nk < 0) nk = 0;
           for (int j = 0; j < nk; j++) {
             double wk = pall[k0 + j] * suffix / l;
             w += wk;

@@ -119,3 +119,29 @@ def test_recorded_p_codes_rebuild_the_pnq_row_sum(tiny, N):
     np.testing.assert_allclose(vals.sum(axis=1), r["l"], rtol=1e-15, atol=0)
     # the group holding the row max (P~ = exp(0) = 1) is never all zero
     assert (vals.max(axis=1) > 0).all()
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_causal_quant_off_equals_masked_softmax_attention(tiny, tau):
+    """Causal masking (row i sees keys 0..i) with quantization off is the textbook masked softmax."""
+    q, k, v = tiny
+    N, d = k.shape
+    rows = np.array([0, 1, 2, 63, 64, 65, 127, 128, 200, N - 1])
+    s = 0.125
+    res = oracle.forward_rows(q[None], k[None], v[None], rows, s, quant=False, tau=tau, causal=True)["out"][0]
+    qr = oracle.rotate_rows(q[rows]).astype(np.float64)
+    kr = oracle.rotate_rows(k).astype(np.float64)
+    S = (qr @ kr.T) * s
+    S[np.arange(N)[None, :] > rows[:, None]] = -np.inf
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    ref = (P / P.sum(axis=1, keepdims=True)) @ v.astype(np.float64)
+    np.testing.assert_allclose(res, ref, rtol=0, atol=1e-5)
+
+
+def test_causal_first_row_sees_only_the_first_key(tiny):
+    """Row 0 under causal masking: one key, P~ = exp(0) = 1 is exact in E2M1, l = 1, so the output
+    is the (quantized) first value row exactly."""
+    q, k, v = tiny
+    res = oracle.forward_rows(q[None], k[None], v[None], np.array([0]), 0.125, causal=True)["out"][0, 0]
+    vq = oracle.prepare_head(q[:1], k, v)[2]
+    np.testing.assert_array_equal(res, vq[0])
