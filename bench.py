@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--causal", action="store_true",
+                    help="causal self-attention; TFLOPS count the visible (query, key) pairs, N(N+1)/2 per head")
     return ap.parse_args()
 
 
@@ -175,6 +177,13 @@ def rank_workload(w, rank: int):
     return inputs.Workload(w.name, 1, w.H, w.N, w.d, w.dtype, w.seed + 1000 * rank)
 
 
+def attention_flops(w, causal: bool) -> float:
+    """The two contractions of one problem: 4 d flops per visible (query, key) pair, N^2 pairs per
+    head, or N(N+1)/2 under causal masking."""
+    pairs = w.N * (w.N + 1) / 2 if causal else float(w.N) * w.N
+    return 4.0 * w.B * w.H * pairs * w.d
+
+
 def whole_job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
     """Throughput of the whole job: every rank's flops over the slowest rank's step time."""
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
@@ -191,7 +200,7 @@ def barrier(dist):
 # ------------------------------------------------------------------------------------------------
 # CPU oracle on a bounded sample
 # ------------------------------------------------------------------------------------------------
-def cpu_oracle_sample(w, target_seconds: float):
+def cpu_oracle_sample(w, target_seconds: float, causal: bool = False):
     """Time the oracle on one head's rotation/quantization plus attention for as many
     query rows as fit the time budget.  Returns (tflops, seconds, description, cores)."""
     import oracle
@@ -213,14 +222,16 @@ def cpu_oracle_sample(w, target_seconds: float):
     sel = np.linspace(0, w.N - 1, nrows).astype(np.int64)
     t2 = time.perf_counter()
     qd, _, _ = oracle.prepare_head(q[sel], k[:32], v[:32])
-    oracle.attention_rows(qd, kd, vd, s, w.key_tile, tau=8.0)
+    oracle.attention_rows(qd, kd, vd, s, w.key_tile, tau=8.0, qpos=sel if causal else None)
     att = time.perf_counter() - t2
     # work: Q/K/V quantization of one head is not attention flops; the metric counts the
     # attention contractions of the sampled rows, timed together with one head's operand prep
-    flops = 4.0 * nrows * w.N * w.d
+    keys = float(np.sum(np.minimum(sel + 1, w.N))) if causal else float(nrows) * w.N
+    flops = 4.0 * keys * w.d
     total = prep + att
     desc = (f"head 0 of {w.name}: rotation+MXFP4 of K and V ({w.N}x{w.d}) and PNQ attention for {nrows} of "
-            f"{w.N} query rows; TFLOPS = 4*rows*N*d / (prep + attention time)")
+            f"{w.N} query rows{' (causal)' if causal else ''}; TFLOPS = 4*(visible query-key pairs)*d / "
+            f"(prep + attention time)")
     return flops / total / 1e12, total, desc, cores
 
 
@@ -239,14 +250,15 @@ def main():
         val = None
         desc = cores = None
         for _ in range(args.warmup + args.steps):
-            val, t, desc, cores = cpu_oracle_sample(w, max(1.0, args.cpu_sample_seconds / max(1, args.steps)))
+            val, t, desc, cores = cpu_oracle_sample(w, max(1.0, args.cpu_sample_seconds / max(1, args.steps)),
+                                                    args.causal)
             times.append(t)
         times = times[args.warmup:]
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                                                "input_dtype": w.dtype},
+                                                "input_dtype": w.dtype, "causal": args.causal},
                 "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc},
                 "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -272,7 +284,7 @@ def main():
     hq, hk, hv = (host_tensor(g[n]) for n in "qkv")
     del g
     q, k, v = (t.to(dev) for t in (hq, hk, hv))
-    opts = binding.Opts()
+    opts = binding.Opts(causal=args.causal)
     scale = float(np.float32(w.d ** -0.5))
     ws = binding.new_workspace(1, w.H, w.N, w.d, opts, dev)
     out = torch.empty(shape, dtype=tdt, device=dev)
@@ -318,7 +330,7 @@ def main():
     total_ms = reduce_max(total_ms, dist)
     attn_ms_max = reduce_max(attn_ms, dist)
     ms_per_step = total_ms / args.steps
-    flops = w.flops  # per rank (B = 1 per rank)
+    flops = attention_flops(w, args.causal)  # per rank (B = 1 per rank)
     value = whole_job_tflops(world, flops, ms_per_step)
     clocks = clk.summary()
 
@@ -360,7 +372,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, t, desc, cores = cpu_oracle_sample(w, args.cpu_sample_seconds)
+        val, t, desc, cores = cpu_oracle_sample(w, args.cpu_sample_seconds, args.causal)
         cpu = {"value": val, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc, "seconds": t}
 
     if rank == 0:
@@ -369,6 +381,7 @@ def main():
                 "vs_baseline": None, "dtype": "fp4(e2m1)+fp32 accumulate, bf16 in/out", "data": "synthetic",
                 "config": {"workload": w.name, "B": world, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
                            "key_tile": 64, "scale_rule": "UOS Qmax=7.25", "pnq": True, "rotate": True,
+                           "causal": args.causal,
                            "rescale_tau": opts.rescale_tau, "parallelism": f"independent problems x{world}",
                            "l2": "inputs (2.3 GB) larger than L2 (126 MB); no flush"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,

@@ -28,7 +28,9 @@
  *  - Arguments are validated before anything is enqueued; an invalid call
  *    returns an error status and enqueues nothing.
  *  - q, k, v, out are contiguous [B, H, N, d] ("BHND") in opts->dtype; out
- *    has the input dtype.  Self-attention without masking, N_q = N_k = N.
+ *    has the input dtype.  Self-attention, N_q = N_k = N, without masking
+ *    unless opts->causal; mxattn_forward_cross takes N_q != N_k and
+ *    mxattn_forward_varlen a token-major packed batch (see there).
  *  - Codes are packed two per byte, element 2i in the LOW nibble, element
  *    2i+1 in the high nibble; bit 3 of a code is the sign (a negative value
  *    that rounds to zero keeps its sign: code 0x8).  Scales are E8M0 bytes
@@ -119,10 +121,16 @@ typedef struct mxattn_opts {
                            /* is checked against it only after a first hardware try_wait */
                            /* returned without the phase); draining in-flight copies and */
                            /* MMAs always gets the default budget.                       */
+  int causal;              /* 1: causal self-attention, query row i sees keys 0..i (an   */
+                           /* autoregressive mask; the pages' video models attend both   */
+                           /* ways and fix none); key tiles past a query tile's diagonal */
+                           /* are skipped.  Self-attention entry points only (varlen:    */
+                           /* within each sequence); cross-attention returns             */
+                           /* MXATTN_ERR_UNSUPPORTED.  0 = full attention.               */
 } mxattn_opts;
 
 /* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
- * key_tile 64, rescale_tau 8, no workspace, default wait budget. */
+ * key_tile 64, rescale_tau 8, no workspace, default wait budget, causal 0. */
 MXATTN_API void mxattn_opts_default(mxattn_opts* opts);
 
 /* Bytes of workspace mxattn_forward needs for this problem (status block plus
@@ -290,6 +298,33 @@ MXATTN_API mxattn_status mxattn_forward_cross(const void* q, const void* k, cons
                                               void* out, void* stream);
 
 /*
+ * Packed batch of variable-length sequences ("varlen"): nseq self-attention
+ * problems of different lengths in one call, e.g. videos of different
+ * durations batched together.  Each sequence is a problem of its own, computed
+ * exactly as mxattn_forward computes one head of it: its V groups of 32 keys
+ * start at its first token, its ragged last tile is masked, and opts->causal
+ * applies within it.  The pages fix no API for this.
+ *  - q, k, v, out: TOKEN-MAJOR [T, H, d] in opts->dtype (T = total tokens,
+ *    row (t, h) at element (t*H + h)*d), 16-byte aligned device pointers.
+ *  - cu_seqlens: DEVICE int32 [nseq + 1], sequence s = tokens cu_seqlens[s] ..
+ *    cu_seqlens[s+1]-1; it must start at 0, never decrease and end at T.
+ *    Empty sequences are allowed.  Being on the device it is checked there: a
+ *    table that breaks the rule makes the pass write nothing and records a
+ *    status that mxattn_get_device_error reports as MXATTN_ERR_INVALID_ARG.
+ *  - nseq in [1, 2^24], H in [1, 65535], d in {64, 128}.
+ *  - Workspace: mxattn_workspace_bytes_varlen(nseq, H, T, d, opts) bytes
+ *    (0 for invalid sizes), 256-byte aligned: status block, the sequences'
+ *    tile table, then the packed operands with every sequence padded to whole
+ *    128-row tiles ((T + 127*nseq)/128 tiles per head are reserved).
+ *  - Four launches on `stream`: the tile table, Q/K rotation+quantization, V
+ *    quantization, the attention.  Other errors as for mxattn_forward.
+ */
+MXATTN_API size_t mxattn_workspace_bytes_varlen(int nseq, int H, int T, int d, const mxattn_opts* opts);
+MXATTN_API mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens,
+                                               int nseq, int H, int T, int d, float softmax_scale,
+                                               const mxattn_opts* opts, void* out, void* stream);
+
+/*
  * mxattn_forward without a caller-provided workspace, for callers that cannot
  * allocate device memory: a process whose memory manager has already reserved
  * the GPU's memory (a cudaMalloc would fail or fragment its pool), or a plain C
@@ -317,7 +352,9 @@ MXATTN_API mxattn_status mxattn_forward_noalloc(const void* q, const void* k, co
 /*
  * Synchronize `stream`, read the workspace status block and clear it.
  * Returns MXATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait since the
- * last call (its output is then undefined), MXATTN_OK otherwise.
+ * last call (its output is then undefined), MXATTN_ERR_INVALID_ARG if a
+ * varlen call found its cu_seqlens table invalid (nothing was written),
+ * MXATTN_OK otherwise.
  */
 MXATTN_API mxattn_status mxattn_get_device_error(const mxattn_opts* opts, void* stream);
 

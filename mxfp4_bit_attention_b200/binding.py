@@ -27,7 +27,7 @@ EXPORTS = (
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
     "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
     "mxattn_workspace_bytes_cross", "mxattn_forward_cross", "mxattn_workspace_bytes_host",
-    "mxattn_forward_host",
+    "mxattn_forward_host", "mxattn_workspace_bytes_varlen", "mxattn_forward_varlen",
 )
 
 
@@ -41,7 +41,8 @@ class COpts(ctypes.Structure):
     _fields_ = [("scale_rule", ctypes.c_int), ("qmax", ctypes.c_float), ("pnq", ctypes.c_int),
                 ("rotate", ctypes.c_int), ("dtype", ctypes.c_int), ("key_tile", ctypes.c_int),
                 ("rescale_tau", ctypes.c_float), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("wait_budget_cycles", ctypes.c_longlong)]
+                ("workspace_bytes", ctypes.c_size_t), ("wait_budget_cycles", ctypes.c_longlong),
+                ("causal", ctypes.c_int)]
 
 
 @dataclass
@@ -53,6 +54,7 @@ class Opts:
     key_tile: int = 64
     rescale_tau: float = 8.0
     wait_budget_cycles: int = 0  # 0: the library's default (about one second)
+    causal: bool = False  # self-attention: query row i sees keys 0..i
 
 
 def lib_path() -> str:
@@ -97,6 +99,8 @@ def load():
         "mxattn_forward_cross": ([P, P, P, i32, i32, i32, i32, i32, f32, PO, P, P], i32),
         "mxattn_workspace_bytes_host": ([i32, i32, i32, i32, PO], sz),
         "mxattn_forward_host": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_workspace_bytes_varlen": ([i32, i32, i32, i32, PO], sz),
+        "mxattn_forward_varlen": ([P, P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -133,6 +137,7 @@ def _copts(o: Opts | None, dtype: int, workspace=None) -> COpts:
     c.scale_rule, c.qmax, c.pnq, c.rotate = int(o.scale_rule), float(o.qmax), int(bool(o.pnq)), int(bool(o.rotate))
     c.dtype, c.key_tile, c.rescale_tau = dtype, int(o.key_tile), float(o.rescale_tau)
     c.wait_budget_cycles = int(o.wait_budget_cycles)
+    c.causal = int(bool(o.causal))
     if workspace is not None:
         c.workspace = ctypes.c_void_p(workspace.data_ptr())
         c.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -312,6 +317,29 @@ def mxattn_forward_cross(q, k, v, softmax_scale=None, opts: Opts | None = None, 
     _check("mxattn_forward_cross", load().mxattn_forward_cross(
         _ptr(q), _ptr(k), _ptr(v), B, H, Nq, Nk, d, float(softmax_scale), ctypes.byref(c), _ptr(out),
         _stream(stream)))
+    return out
+
+
+def mxattn_forward_varlen(q, k, v, cu_seqlens, softmax_scale=None, opts: Opts | None = None, out=None,
+                          workspace=None, stream=None):
+    """Packed batch of variable-length sequences: q, k, v, out token-major [T, H, d]; cu_seqlens an
+    int32 device tensor [nseq + 1] (sequence s = tokens cu_seqlens[s] .. cu_seqlens[s+1]-1).  An
+    invalid cu_seqlens is reported by mxattn_get_device_error (MXATTN_ERR_INVALID_ARG)."""
+    import torch
+    T, H, d = q.shape
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise TypeError("cu_seqlens must be a contiguous 1-D int32 tensor")
+    nseq = cu_seqlens.numel() - 1
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    out = out if out is not None else torch.empty_like(q)
+    if workspace is None:
+        nbytes = load().mxattn_workspace_bytes_varlen(nseq, H, T, d, ctypes.byref(_copts(opts, _dtype_code(q))))
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=q.device)
+    c = _copts(opts, _dtype_code(q), workspace)
+    _check("mxattn_forward_varlen", load().mxattn_forward_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, H, T, d, float(softmax_scale), ctypes.byref(c),
+        _ptr(out), _stream(stream)))
     return out
 
 

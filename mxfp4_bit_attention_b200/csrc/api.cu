@@ -61,6 +61,7 @@ mxattn_status check_opts(const mxattn_opts* o) {
   if (!(o->rescale_tau >= 0.f && std::isfinite(o->rescale_tau))) return MXATTN_ERR_INVALID_ARG;
   if (o->key_tile != 64) return o->key_tile == 128 ? MXATTN_ERR_UNSUPPORTED : MXATTN_ERR_INVALID_ARG;
   if (o->wait_budget_cycles < 0) return MXATTN_ERR_INVALID_ARG;
+  if (o->causal != 0 && o->causal != 1) return MXATTN_ERR_INVALID_ARG;
   return MXATTN_OK;
 }
 
@@ -110,6 +111,7 @@ void mxattn_opts_default(mxattn_opts* o) {
   o->workspace = nullptr;
   o->workspace_bytes = 0;
   o->wait_budget_cycles = 0;
+  o->causal = 0;
 }
 
 size_t mxattn_qk_codes_bytes(int B, int H, int N, int d) {
@@ -176,7 +178,7 @@ mxattn_status quant_qk(const void* q, const void* k, int B, int H, int Nq, int N
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_codes) || !aligned16(k_codes)) return MXATTN_ERR_INVALID_ARG;
-  QKQuantArgs a;
+  QKQuantArgs a{};
   a.q = q;
   a.k = k;
   a.q_codes = q_codes;
@@ -209,7 +211,7 @@ mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mx
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
   if (!aligned16(v) || !aligned16(v_codes)) return MXATTN_ERR_INVALID_ARG;
-  VQuantArgs a;
+  VQuantArgs a{};
   a.v = v;
   a.v_codes = v_codes;
   a.v_scales = v_scales;
@@ -231,12 +233,13 @@ mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const u
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
+  if (o->causal && Nq != Nk) return MXATTN_ERR_UNSUPPORTED;
   st = check_workspace(o, kStatusBytes);
   if (st != MXATTN_OK) return st;
   const void* ptrs[] = {q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, out};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MXATTN_ERR_INVALID_ARG;
-  AttnArgs a;
+  AttnArgs a{};
   a.q_codes = q_codes;
   a.q_scales = q_scales;
   a.k_codes = k_codes;
@@ -253,6 +256,7 @@ mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const u
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
+  a.causal = o->causal;
   a.dump = nullptr;
   a.dump_bh = a.dump_qt = -1;
   return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
@@ -287,7 +291,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   if (st != MXATTN_OK) return st;
   st = check_workspace(o, kStatusBytes);
   if (st != MXATTN_OK) return st;
-  AttnArgs a;
+  AttnArgs a{};
   a.q_codes = q_codes;
   a.q_scales = q_scales;
   a.k_codes = k_codes;
@@ -304,6 +308,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
+  a.causal = o->causal;
   a.dump = dump;
   a.dump_bh = dump_bh;
   a.dump_qt = dump_qt;
@@ -344,6 +349,7 @@ mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, 
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
+  if (o->causal) return MXATTN_ERR_UNSUPPORTED;  // no query/key position correspondence
   const Carve c = carve(B, H, Nq, Nk, d);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
@@ -355,6 +361,127 @@ mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, 
   if (st != MXATTN_OK) return st;
   return attention(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes, ws + c.v_scales,
                    B, H, Nq, Nk, d, softmax_scale, o, out, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Packed varlen batch: nseq sequences, T tokens, token-major [T, H, d].  Every sequence is padded
+// to whole 128-row tiles in the packed operands; sum over s of ceil(len_s / 128) is at most
+// (T + 127 nseq) / 128 tiles per head, the stride the packing reserves.
+constexpr int kMaxVarlenSeqs = 1 << 24;
+
+bool varlen_sizes_ok(int nseq, int H, int T, int d, int64_t* tiles_per_head) {
+  if (nseq < 1 || nseq > kMaxVarlenSeqs || H < 1 || H > 65535 || T < 1 || (d != 64 && d != 128)) return false;
+  const int64_t tph = ((int64_t)T + 127 * (int64_t)nseq) / 128;
+  if ((int64_t)H * 2 * tph >= ((int64_t)1 << 31)) return false;  // blocks of the V quantizer
+  *tiles_per_head = tph;
+  return true;
+}
+
+struct VarlenCarve {
+  size_t tile_off, q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, total;
+};
+
+VarlenCarve carve_varlen(int nseq, int H, int64_t tph, int d) {
+  VarlenCarve c;
+  const size_t codes = (size_t)H * tph * 128 * (d / 2), scales = (size_t)H * tph * 512;
+  size_t off = kStatusBytes;
+  c.tile_off = off; off = align256(off + ((size_t)nseq + 1) * sizeof(int));
+  c.q_codes = off; off = align256(off + codes);
+  c.q_scales = off; off = align256(off + scales);
+  c.k_codes = off; off = align256(off + codes);
+  c.k_scales = off; off = align256(off + scales);
+  c.v_codes = off; off = align256(off + codes);  // 2 tph tiles of 64 keys x d channels x 32 bytes
+  c.v_scales = off; off = align256(off + scales);
+  c.total = off;
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mxattn_workspace_bytes_varlen(int nseq, int H, int T, int d, const mxattn_opts* opts) {
+  (void)opts;
+  int64_t tph;
+  if (!varlen_sizes_ok(nseq, H, T, d, &tph)) return 0;
+  return carve_varlen(nseq, H, tph, d).total;
+}
+
+mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, int nseq,
+                                    int H, int T, int d, float softmax_scale, const mxattn_opts* o, void* out,
+                                    void* stream) {
+  int64_t tph;
+  if (!varlen_sizes_ok(nseq, H, T, d, &tph)) return MXATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !cu_seqlens) return MXATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
+  mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  const VarlenCarve c = carve_varlen(nseq, H, tph, d);
+  st = check_workspace(o, c.total);
+  if (st != MXATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return MXATTN_ERR_INVALID_ARG;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  int* tile_off = reinterpret_cast<int*>(ws + c.tile_off);
+  const cudaStream_t s = as_stream(stream);
+  const Varlen vl{cu_seqlens, tile_off, nseq, (int)tph};
+  st = launched(launch_varlen_tiles(cu_seqlens, nseq, T, tile_off, status, s));
+  if (st != MXATTN_OK) return st;
+  ScaleRule rule;
+  make_rule(o, &rule);
+
+  QKQuantArgs qa{};
+  qa.q = q;
+  qa.k = k;
+  qa.q_codes = ws + c.q_codes;
+  qa.q_scales = ws + c.q_scales;
+  qa.k_codes = ws + c.k_codes;
+  qa.k_scales = ws + c.k_scales;
+  qa.BH = H;
+  qa.N = qa.Nk = T;
+  qa.rotate = o->rotate;
+  qa.hadamard_scale = (float)(1.0 / std::sqrt((double)d));
+  qa.rule = rule;
+  qa.vl = vl;
+  st = launched(launch_rotate_quant_qk(qa, d, o->dtype, s));
+  if (st != MXATTN_OK) return st;
+
+  VQuantArgs va{};
+  va.v = v;
+  va.v_codes = ws + c.v_codes;
+  va.v_scales = ws + c.v_scales;
+  va.BH = H;
+  va.N = T;
+  va.rule = rule;
+  va.vl = vl;
+  st = launched(launch_quant_v(va, d, o->dtype, s));
+  if (st != MXATTN_OK) return st;
+
+  AttnArgs a{};
+  a.q_codes = ws + c.q_codes;
+  a.q_scales = ws + c.q_scales;
+  a.k_codes = ws + c.k_codes;
+  a.k_scales = ws + c.k_scales;
+  a.v_codes = ws + c.v_codes;
+  a.v_scales = ws + c.v_scales;
+  a.out = out;
+  a.status = status;
+  a.BH = H;
+  a.N = a.Nk = T;
+  a.causal = o->causal;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+  a.tau = o->rescale_tau;
+  a.pnq = o->pnq;
+  a.rule = rule;
+  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
+  a.dump = nullptr;
+  a.dump_bh = a.dump_qt = -1;
+  a.vl = vl;
+  return launched(launch_attention(a, d, o->dtype, s));
 }
 
 }  // extern "C"
@@ -533,7 +660,7 @@ mxattn_status mxattn_get_device_error(const mxattn_opts* o, void* stream) {
   if (words[0] == 0) return MXATTN_OK;
   if (cudaMemsetAsync(o->workspace, 0, kStatusBytes, s) != cudaSuccess) return MXATTN_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MXATTN_ERR_CUDA;
-  return MXATTN_ERR_TIMEOUT;
+  return words[0] == kStatusBadSeqlens ? MXATTN_ERR_INVALID_ARG : MXATTN_ERR_TIMEOUT;
 }
 
 const char* mxattn_status_string(mxattn_status s) {

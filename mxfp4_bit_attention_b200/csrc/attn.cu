@@ -38,6 +38,9 @@ namespace mxattn {
 
 constexpr int kBM = 128;        // query rows per CTA
 constexpr int kBN = 64;         // keys per tile
+// Kernel variants: the fixed-shape full-attention pass (timed), the same with the diagnostic dump
+// of one CTA, and the masked variant (causal masking and/or a packed varlen batch).
+enum { kModeFull = 0, kModeDump = 1, kModeMasked = 2 };
 constexpr int kStages = 4;      // K/V shared-memory ring depth
 constexpr int kSfSlots = 3;     // K/V scale-factor slots in TMEM (reuse distance 3 tiles)
 // Warps 0-3 run the softmax (warp w reads TMEM lanes 32w..32w+31); the producer and the two MMA
@@ -182,19 +185,51 @@ __device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, i
   }
 }
 
-template <int D, int DT, bool PNQ, bool DUMP>
+template <int D, int DT, bool PNQ, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
   using L = Layout<D>;
+  constexpr bool DUMP = MODE == kModeDump;
+  constexpr bool MASKED = MODE == kModeMasked;
   constexpr int NV = PNQ ? D + kOnesRows : D;  // N of the PV MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T128 = (a.N + 127) / 128;   // query tiles of a head
-  const int T128k = (a.Nk + 127) / 128; // 128-key operand tiles of a head
-  const int T64 = (a.Nk + 63) / 64;     // 64-key tiles swept by the CTA
-  const int qt = blockIdx.x;
+  const bool causal = MASKED && a.causal;
+  // The problem of this CTA: query tile qt (rows 128qt..) of head bh, with Nq query rows and Nk
+  // keys; the packed operand tiles it reads and where its output rows go.  Under causal masking
+  // the longest query tiles (the last ones) are launched first, so that the short ones fill in
+  // behind them.
   const int bh = blockIdx.y;
+  int Nq = a.N, Nk = a.Nk, qt;
+  size_t q_tile, k_tile0, v_tile0;  // Q tile, first 128-key K tile / scale atom, first 64-key V tile
+  size_t out_row0, out_step;        // output element offset of query row 0, and per row
+  if (MASKED && a.vl.cu_seqlens != nullptr) {
+    // packed varlen batch: blockIdx.x runs over the tiles of all sequences; token-major [T, H, d]
+    const int g = causal ? a.vl.tiles_per_head - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    if (g >= __ldg(a.vl.tile_off + a.vl.nseq)) return;  // past the last sequence: the whole CTA
+    const int sq = varlen_sequence(a.vl, g);
+    const int start = __ldg(a.vl.cu_seqlens + sq);
+    Nq = Nk = __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    const int t0 = __ldg(a.vl.tile_off + sq);
+    qt = g - t0;
+    q_tile = (size_t)bh * a.vl.tiles_per_head + g;
+    k_tile0 = (size_t)bh * a.vl.tiles_per_head + t0;
+    v_tile0 = 2 * k_tile0;
+    out_row0 = ((size_t)start * a.BH + bh) * D;
+    out_step = (size_t)a.BH * D;
+  } else {
+    const int T128 = (a.N + 127) / 128;
+    qt = causal ? T128 - 1 - (int)blockIdx.x : (int)blockIdx.x;
+    q_tile = (size_t)bh * T128 + qt;
+    k_tile0 = (size_t)bh * ((a.Nk + 127) / 128);
+    v_tile0 = (size_t)bh * ((a.Nk + 63) / 64);
+    out_row0 = (size_t)bh * a.N * D;
+    out_step = D;
+  }
+  const int T64 = (Nk + 63) / 64;  // 64-key tiles of the problem
+  // tiles the CTA sweeps: all, or under causal masking those up to its diagonal
+  const int TJ = causal ? (2 * qt + 2 < T64 ? 2 * qt + 2 : T64) : T64;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::ABORT);
   __shared__ int never;  // a flag nothing sets: drains ignore the abort flag
   auto bar = [&](int i) -> uint32_t { return sb + L::BARS + 8 * i; };
@@ -243,24 +278,23 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     if (lane == 0) {
       bool ok = true;
       int issued = 0;
-      const size_t qtile = (size_t)bh * T128 + qt;
       mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES + 512);
-      bulk_g2s(sb + L::Q_CODES, a.q_codes + qtile * (size_t)L::Q_BYTES, L::Q_BYTES, bar(L::B_Q));
-      bulk_g2s(sb + L::SF_Q, a.q_scales + qtile * 512, 512, bar(L::B_Q));
-      for (int j = 0; j < T64; j++) {
+      bulk_g2s(sb + L::Q_CODES, a.q_codes + q_tile * (size_t)L::Q_BYTES, L::Q_BYTES, bar(L::B_Q));
+      bulk_g2s(sb + L::SF_Q, a.q_scales + q_tile * 512, 512, bar(L::B_Q));
+      for (int j = 0; j < TJ; j++) {
         const int s = j % kStages;
         if (j >= kStages) {
           ok = mbar_wait(bar(L::B_KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, a.wait_budget);
           if (!ok) break;
         }
         const uint32_t fb = bar(L::B_KV_FULL + s);
-        const size_t t128 = (size_t)bh * T128k + j / 2;
+        const size_t t128 = k_tile0 + j / 2;
         mbar_arrive_expect_tx(fb, L::K_BYTES + L::V_BYTES + 1024);
         bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES,
                  a.k_codes + (t128 * kBM + (j % 2) * kBN) * (size_t)(D / 2), L::K_BYTES, fb);
         bulk_g2s(sb + L::SF_K + s * 512, a.k_scales + t128 * 512, 512, fb);
         bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES + L::K_BYTES,
-                 a.v_codes + ((size_t)bh * T64 + j) * (size_t)L::V_BYTES, L::V_BYTES, fb);
+                 a.v_codes + (v_tile0 + j) * (size_t)L::V_BYTES, L::V_BYTES, fb);
         bulk_g2s(sb + L::SF_V + s * 512, a.v_scales + t128 * 512, 512, fb);
         issued = j + 1;
       }
@@ -283,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       if (leader) tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
       __syncwarp();
       const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
-      for (int j = 0; j < T64; j++) {
+      for (int j = 0; j < TJ; j++) {
         const int s = j % kStages, f = j % kSfSlots;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
         if (!ok) break;
@@ -329,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
     __syncwarp();
     bool ok = true;
-    for (int jp = 0; jp < T64; jp++) {
+    for (int jp = 0; jp < TJ; jp++) {
       const int sp = jp % kStages, fp = jp % kSfSlots, pb = jp & 1;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget));
       if (!ok) break;
@@ -371,6 +405,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     const float c = a.scale_log2;
     const bool dumping = DUMP && bh == a.dump_bh && qt == a.dump_qt;
     const DumpLayout dl(D, T64);
+    // keys this row sees: all Nk, or under causal masking those up to its own position
+    const int kmax = causal ? (qt * kBM + row + 1 < Nk ? qt * kBM + row + 1 : Nk) : Nk;
     float sm = -INFINITY;  // running max of S used for the exponent (raw MMA units)
     float m2 = -INFINITY;  // the same in log2 units, fl32(sm * c)
     float l = 0.f;         // direct placement only (PNQ keeps l in O~ column D)
@@ -402,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
       }
 
-      const int valid = FULL ? kBN : a.Nk - j * kBN;
+      const int valid = FULL ? kBN : kmax - j * kBN;  // this row's keys in the tile (may be <= 0)
       float gmax[2];
       if (FULL) {
         gmax[0] = group_max<false>(s0, 0, valid);
@@ -440,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         group_codes<true, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
       }
       // test S(j+1) now, so that the test's latency overlaps the stores below
-      s_ready = j + 1 < T64 && mbar_test(bar(L::B_S_FULL), (j + 1) & 1);
+      s_ready = j + 1 < TJ && mbar_test(bar(L::B_S_FULL), (j + 1) & 1);
       if (!PNQ) {
         float lsum = 0.f;
 #pragma unroll
@@ -502,15 +538,22 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
       return true;
     };
-    const int full_tiles = (a.Nk % kBN == 0) ? T64 : T64 - 1;
+    // tiles every row of the CTA sees in full, then the masked ones (the ragged last tile of the
+    // keys; under causal masking the two diagonal tiles)
+    int full_tiles = (Nk % kBN == 0) ? T64 : T64 - 1;
+    if (causal && full_tiles > 2 * qt) full_tiles = 2 * qt;
     for (int j = 0; ok && j < full_tiles; j++) ok = tile(j, std::true_type{});
-    if (ok && full_tiles < T64) ok = tile(T64 - 1, std::false_type{});
-    if (ok && T64 >= 2) {  // the last two PV MMAs, one on each O_DONE barrier
-      ok = mbar_wait(bar(L::B_O_DONE + (T64 & 1)), ((T64 - 2) >> 1) & 1, abort_flag, a.wait_budget);
+    if (MASKED) {
+      for (int j = full_tiles; ok && j < TJ; j++) ok = tile(j, std::false_type{});
+    } else if (ok && full_tiles < T64) {
+      ok = tile(T64 - 1, std::false_type{});  // the ragged last tile
+    }
+    if (ok && TJ >= 2) {  // the last two PV MMAs, one on each O_DONE barrier
+      ok = mbar_wait(bar(L::B_O_DONE + (TJ & 1)), ((TJ - 2) >> 1) & 1, abort_flag, a.wait_budget);
       ok = __all_sync(0xFFFFFFFFu, ok);
     }
     if (ok) {
-      ok = mbar_wait(bar(L::B_O_DONE + ((T64 - 1) & 1)), ((T64 - 1) >> 1) & 1, abort_flag, a.wait_budget);
+      ok = mbar_wait(bar(L::B_O_DONE + ((TJ - 1) & 1)), ((TJ - 1) >> 1) & 1, abort_flag, a.wait_budget);
       ok = __all_sync(0xFFFFFFFFu, ok);
     }
     if (ok) {
@@ -524,8 +567,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
       const float inv_l = 1.f / l;
       const int qrow = qt * kBM + row;
-      const bool store = qrow < a.N;
-      const size_t obase = ((size_t)bh * a.N + (store ? qrow : 0)) * D;
+      const bool store = qrow < Nq;
+      const size_t obase = out_row0 + (size_t)(store ? qrow : 0) * out_step;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; cc++) {
         uint32_t o[32];
@@ -579,11 +622,16 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
 template <int D, int DT, bool PNQ>
 static cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
   using L = Layout<D>;
-  // the diagnostic dump is a separate instantiation, so the timed kernel carries none of it
-  auto kern = a.dump != nullptr ? mxattn_fwd_kernel<D, DT, PNQ, true> : mxattn_fwd_kernel<D, DT, PNQ, false>;
+  // the diagnostic dump and the masking are separate instantiations, so the timed kernel carries
+  // none of them
+  const bool masked = a.causal || a.vl.cu_seqlens != nullptr;
+  auto kern = a.dump != nullptr ? mxattn_fwd_kernel<D, DT, PNQ, kModeDump>
+              : masked          ? mxattn_fwd_kernel<D, DT, PNQ, kModeMasked>
+                                : mxattn_fwd_kernel<D, DT, PNQ, kModeFull>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_SMEM);
   if (err != cudaSuccess) return err;
-  dim3 grid((unsigned)((a.N + kBM - 1) / kBM), (unsigned)a.BH);
+  const unsigned qtiles = a.vl.cu_seqlens != nullptr ? (unsigned)a.vl.tiles_per_head : (unsigned)((a.N + kBM - 1) / kBM);
+  dim3 grid(qtiles, (unsigned)a.BH);
   kern<<<grid, kThreads, L::DYN_SMEM, s>>>(a);
   return cudaGetLastError();
 }

@@ -10,6 +10,29 @@ namespace mxattn {
 
 enum { kBF16 = 0, kFP32 = 1 };
 
+// A packed batch of variable-length sequences ("varlen"): inputs and outputs are token-major
+// [T, H, d]; sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 and is padded to whole
+// 128-row tiles in the packed operands, where it starts at tile tile_off[s] of each head's
+// tiles_per_head tiles.  cu_seqlens == nullptr: the fixed-length [B, H, N, d] layout.
+struct Varlen {
+  const int* cu_seqlens;  // [nseq + 1] device
+  const int* tile_off;    // [nseq + 1] device, written by the tile-table kernel
+  int nseq;
+  int tiles_per_head;
+};
+
+// Sequence owning packed tile g (tile_off[nseq] > g): the last s with tile_off[s] <= g (empty
+// sequences own no tile and are skipped).
+__device__ __forceinline__ int varlen_sequence(const Varlen& v, int g) {
+  int lo = 0, hi = v.nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(v.tile_off + mid) <= g) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 struct QKQuantArgs {
   const void* q;
   const void* k;
@@ -17,19 +40,21 @@ struct QKQuantArgs {
   uint8_t* q_scales;
   uint8_t* k_codes;
   uint8_t* k_scales;
-  int BH, N;             // N: tokens of Q
+  int BH, N;             // N: tokens of Q (varlen: BH = H, N = T)
   int Nk;                // tokens of K (= N for self-attention)
   int rotate;
   float hadamard_scale;  // fl32(1/sqrt(d))
   ScaleRule rule;
+  Varlen vl;
 };
 
 struct VQuantArgs {
   const void* v;
   uint8_t* v_codes;
   uint8_t* v_scales;
-  int BH, N;
+  int BH, N;             // varlen: BH = H, N = T
   ScaleRule rule;
+  Varlen vl;
 };
 
 struct PlainQuantArgs {
@@ -65,6 +90,7 @@ struct AttnArgs {
   int* status;           // workspace status block (error word at [0], detail at [1..3])
   int BH, N;             // N: query rows per head
   int Nk;                // keys (and values) per head (= N for self-attention)
+  int causal;            // self-attention only: query row i sees keys 0..i
   float scale_log2;      // softmax_scale * log2(e)
   float tau;             // lazy max threshold, log2 units
   int pnq;
@@ -72,6 +98,7 @@ struct AttnArgs {
   long long wait_budget; // SM clock cycles a bounded wait may spin before giving up
   uint8_t* dump;         // optional diagnostic dump of one CTA (layout: see dump_layout below)
   int dump_bh, dump_qt;
+  Varlen vl;             // varlen: BH = H, N = Nk = T
 };
 
 // Diagnostic dump of the CTA (dump_bh, dump_qt), byte offsets for head dim D and T64 key tiles:
@@ -98,8 +125,9 @@ struct DumpLayout {
   }
 };
 
-// Status words written by a kernel whose bounded wait expired.
-enum { kStatusTimeout = 0x54494D45 /* 'TIME' */ };
+// Status words: a kernel whose bounded wait expired; sequence offsets that are not a partition
+// of the packed tokens.
+enum { kStatusTimeout = 0x54494D45 /* 'TIME' */, kStatusBadSeqlens = 0x5345514C /* 'SEQL' */ };
 
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s);
@@ -107,5 +135,6 @@ cudaError_t launch_quant_plain(const PlainQuantArgs& a, int dtype, cudaStream_t 
 cudaError_t launch_qmax_sweep(const SweepArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_fp4_mma_probe(int ctas, int iters, int n, int* status, cudaStream_t s);
+cudaError_t launch_varlen_tiles(const int* cu_seqlens, int nseq, int T, int* tile_off, int* status, cudaStream_t s);
 
 }  // namespace mxattn

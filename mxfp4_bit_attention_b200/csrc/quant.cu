@@ -45,7 +45,8 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid,
 // One thread per MX group (32 consecutive elements of a row, four 16-byte loads in flight), D/32
 // threads per row: butterfly stages h = 1..16 run inside the thread, h = 32 and 64 across the
 // row's threads by shuffles, in the order h = 1, 2, ..., D/2; the group max is the thread's own.
-// Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K.
+// Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K;
+// varlen: over H * tiles_per_head * 128 padded rows, each tile belonging to one sequence.
 // ------------------------------------------------------------------------------------------------
 template <int D, int DT>
 __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
@@ -55,19 +56,36 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
   const int g = t % TPR;                     // group (and 16-byte code chunk) within the row
   const int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;   // padded row id
   const int Nt = blockIdx.y == 0 ? a.N : a.Nk;  // tokens of this tensor
-  const int64_t T128 = (Nt + 127) / 128;
+  const bool vl = a.vl.cu_seqlens != nullptr;
+  const int64_t T128 = vl ? a.vl.tiles_per_head : (Nt + 127) / 128;  // 128-row tiles per head
   const int64_t total = (int64_t)a.BH * T128 * 128;
-  const bool row_ok = prow < total;          // a row's threads are adjacent lanes of one warp
+  bool row_ok = prow < total;                // a row's threads are adjacent lanes of one warp
   const int64_t bh = prow / (T128 * 128);
-  const int tok = (int)(prow % (T128 * 128));
-  const bool valid = row_ok && tok < Nt;
+  const int r = (int)(prow % 128);           // row within its tile
+  const int64_t tile = prow / 128;           // packed tile (bh * T128 + tile within the head)
+  bool valid;
+  int64_t src_row;                           // row of the [rows, D] source
+  if (vl) {
+    // the tile's sequence and the row's token within it; tiles past the last sequence's are unused
+    const int gt = (int)(tile - bh * T128);
+    row_ok = row_ok && gt < __ldg(a.vl.tile_off + a.vl.nseq);
+    const int sq = row_ok ? varlen_sequence(a.vl, gt) : 0;
+    const int start = __ldg(a.vl.cu_seqlens + sq);
+    const int n = (gt - __ldg(a.vl.tile_off + sq)) * 128 + r;
+    valid = row_ok && n < __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    src_row = ((int64_t)start + n) * a.BH + bh;  // token-major [T, H, d]
+  } else {
+    const int tok = (int)(prow % (T128 * 128));
+    valid = row_ok && tok < Nt;
+    src_row = (int64_t)bh * Nt + tok;
+  }
 
   const void* src = blockIdx.y == 0 ? a.q : a.k;
   uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
   uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
 
   float v[32];
-  const int64_t base = ((int64_t)bh * Nt + (valid ? tok : 0)) * D + g * 32;
+  const int64_t base = (valid ? src_row : 0) * D + g * 32;
 #pragma unroll
   for (int c = 0; c < 4; c++) load8<DT>(src, base + c * 8, valid, *reinterpret_cast<float(*)[8]>(v + 8 * c));
 
@@ -127,8 +145,6 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
                       __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
                       __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
   if (!row_ok) return;
-  const int r = tok % 128;
-  const int64_t tile = bh * T128 + tok / 128;
   const int s = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
   uint8_t* rowp = codes + (tile * 128 + r) * (D / 2);
   *reinterpret_cast<uint4*>(rowp + ((g ^ s) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -141,14 +157,41 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
 // V: quantization along keys (32 consecutive tokens per channel) into the packed V operand
 // layout.  One block per (head, 64-key tile): the tile is staged through shared memory as
 // fp32 [64][D+1], then thread (channel c, half h) quantizes keys 32h..32h+31 of channel c.
+// Varlen: blocks over (head, 64-key tile of the packed tiles); each sequence's groups start at
+// its first token, and a sequence's tiles past its own keys are left unwritten.
 // ------------------------------------------------------------------------------------------------
 template <int D, int DT>
 __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
   __shared__ float tile[64][D + 1];
-  const int T64 = (a.N + 63) / 64;
-  const int T128 = (a.N + 127) / 128;
-  const int bh = blockIdx.x / T64;
-  const int j = blockIdx.x % T64;
+  const bool vl = a.vl.cu_seqlens != nullptr;
+  int N = a.N;                                  // keys of this block's sequence
+  int T64, bh, j;                               // its 64-key tiles, head, and this tile among them
+  int64_t src_row0, src_stride;                 // source row of key 0 and the row step per key
+  int64_t vtile, atom_tile;                     // packed 64-key code tile and 128-key scale atom
+  if (vl) {
+    const int per_head = 2 * a.vl.tiles_per_head;
+    bh = blockIdx.x / per_head;
+    const int jg = blockIdx.x % per_head;
+    if (jg / 2 >= __ldg(a.vl.tile_off + a.vl.nseq)) return;
+    const int sq = varlen_sequence(a.vl, jg / 2);
+    const int start = __ldg(a.vl.cu_seqlens + sq);
+    N = __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    T64 = (N + 63) / 64;
+    j = jg - 2 * __ldg(a.vl.tile_off + sq);
+    if (j >= T64) return;                       // the unused odd half of a sequence's last atom
+    src_row0 = (int64_t)start * a.BH + bh;
+    src_stride = a.BH;
+    vtile = (int64_t)bh * per_head + jg;
+    atom_tile = (int64_t)bh * a.vl.tiles_per_head + jg / 2;
+  } else {
+    T64 = (N + 63) / 64;
+    bh = blockIdx.x / T64;
+    j = blockIdx.x % T64;
+    src_row0 = (int64_t)bh * N;
+    src_stride = 1;
+    vtile = (int64_t)bh * T64 + j;
+    atom_tile = (int64_t)bh * ((N + 127) / 128) + j / 2;
+  }
   const int t = threadIdx.x;
   // stage: 64 tokens x D values, 8 values per thread-iteration
   constexpr int VEC_PER_ROW = D / 8;
@@ -158,7 +201,7 @@ __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
     const int row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
     const int tok = j * 64 + row;
     float v[8];
-    load8<DT>(a.v, ((int64_t)bh * a.N + (tok < a.N ? tok : 0)) * D + cv * 8, tok < a.N, v);
+    load8<DT>(a.v, (src_row0 + (tok < N ? tok : 0) * src_stride) * D + cv * 8, tok < N, v);
 #pragma unroll
     for (int i = 0; i < 8; i++) tile[row][cv * 8 + i] = v[i];
   }
@@ -179,9 +222,9 @@ __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
                         __fmul_rn(tile[b + 4][c], inv), __fmul_rn(tile[b + 5][c], inv),
                         __fmul_rn(tile[b + 6][c], inv), __fmul_rn(tile[b + 7][c], inv));
     }
-    uint8_t* dst = a.v_codes + (((int64_t)bh * T64 + j) * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+    uint8_t* dst = a.v_codes + (vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
     *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    uint8_t* atom = a.v_scales + ((int64_t)bh * T128 + j / 2) * 512;
+    uint8_t* atom = a.v_scales + atom_tile * 512;
     atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
     if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
     // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
@@ -239,7 +282,8 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
 // Launchers
 // ------------------------------------------------------------------------------------------------
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
-  const int64_t rows = (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
+  const int64_t rows = a.vl.cu_seqlens != nullptr ? (int64_t)a.BH * a.vl.tiles_per_head * 128
+                                                  : (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
   const int rows_per_block = 256 / (D / 32);
   dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
   if (D == 128 && dtype == kBF16) rotate_quant_qk_kernel<128, kBF16><<<grid, 256, 0, s>>>(a);
@@ -250,7 +294,8 @@ cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaS
 }
 
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s) {
-  const unsigned blocks = (unsigned)((int64_t)a.BH * ((a.N + 63) / 64));
+  const unsigned blocks = (unsigned)((int64_t)a.BH * (a.vl.cu_seqlens != nullptr ? 2 * (int64_t)a.vl.tiles_per_head
+                                                                                 : (a.N + 63) / 64));
   if (D == 128 && dtype == kBF16) quant_v_kernel<128, kBF16><<<blocks, 256, 0, s>>>(a);
   else if (D == 128) quant_v_kernel<128, kFP32><<<blocks, 256, 0, s>>>(a);
   else if (dtype == kBF16) quant_v_kernel<64, kBF16><<<blocks, 256, 0, s>>>(a);

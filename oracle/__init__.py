@@ -246,6 +246,34 @@ def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=
     return res
 
 
+def forward_varlen(q, k, v, cu_seqlens, rows, softmax_scale, causal=False, with_l=False, **kw):
+    """Attention over a packed batch of variable-length sequences: sequence s holds tokens
+    cu_seqlens[s] .. cu_seqlens[s+1]-1 and attends only to its own tokens, as an attention problem
+    of its own (its V groups of 32 keys start at its first token).  This is the definition of a
+    packed batch: each sequence is handed to forward_rows on its own.
+
+    q, k, v: fp32 arrays [T, H, d] (token-major packing).  rows: global token indices.
+    Keyword arguments go to forward_rows.  Returns out [len(rows), H, d] (fp64), and with with_l
+    also the row sums l [len(rows), H] (in units of the row's running maximum).
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    T, H, d = q.shape
+    assert cu[0] == 0 and cu[-1] == T and (np.diff(cu) >= 0).all()
+    out = np.zeros((len(rows), H, d))
+    ls = np.zeros((len(rows), H))
+    seq = np.searchsorted(cu, rows, side="right") - 1
+    for s in np.unique(seq):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        sel = np.nonzero(seq == s)[0]
+        per_head = lambda x: np.ascontiguousarray(x[lo:hi].transpose(1, 0, 2))
+        res = forward_rows(per_head(q), per_head(k), per_head(v), rows[sel] - lo, softmax_scale,
+                           causal=causal, **kw)
+        out[sel] = res["out"].transpose(1, 0, 2)
+        ls[sel] = res["l"].T
+    return (out, ls) if with_l else out
+
+
 # ----------------------------------------------------------------------------------------------
 # Scale-rule diagnostic: per-block Qmax sweep
 # ----------------------------------------------------------------------------------------------

@@ -36,6 +36,7 @@ def test_host_only_calls(lib):
     assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 64)
     assert abs(o.qmax - 7.25) < 1e-7 and abs(o.rescale_tau - 8.0) < 1e-7
     assert o.wait_budget_cycles == 0  # the library's default budget
+    assert o.causal == 0
     assert lib.mxattn_qk_codes_bytes(1, 2, 200, 128) == 2 * 2 * 128 * 64
     assert lib.mxattn_qk_scales_bytes(1, 2, 200, 128) == 2 * 2 * 512
     assert lib.mxattn_v_codes_bytes(1, 2, 200, 128) == 2 * 4 * 128 * 32
@@ -50,6 +51,12 @@ def test_host_only_calls(lib):
     # staging for two chunks of 4 heads, far below the 2.3 GB of all 40 heads' bf16 inputs
     assert 0 < lib.mxattn_workspace_bytes_host(1, 40, 75600, 128, ctypes.byref(o)) < 3 * 40 * 75600 * 128 * 2 // 3
     assert lib.mxattn_workspace_bytes_host(1, 1, 0, 128, ctypes.byref(o)) == 0
+    # varlen: (T + 127 nseq) / 128 tiles per head reserved; one sequence packs like B = 1
+    one = lib.mxattn_workspace_bytes_varlen(1, 4, 1000, 128, ctypes.byref(o))
+    assert one >= lib.mxattn_workspace_bytes(1, 4, 1000, 128, ctypes.byref(o))
+    assert lib.mxattn_workspace_bytes_varlen(3, 4, 1000, 128, ctypes.byref(o)) > one
+    assert lib.mxattn_workspace_bytes_varlen(0, 4, 1000, 128, ctypes.byref(o)) == 0
+    assert lib.mxattn_workspace_bytes_varlen(2, 4, 1000, 96, ctypes.byref(o)) == 0
     assert lib.mxattn_status_string(5) == b"MXATTN_ERR_TIMEOUT"
 
 
@@ -75,6 +82,21 @@ def test_validation_rejects_before_enqueue(lib):
     o.wait_budget_cycles = -5
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
     o.wait_budget_cycles = 0
+    o.causal = 2
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
+    o.causal = 1  # causal masking needs a query/key position correspondence
+    assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 64, 0.1, P, fake, None) == 2
+    assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 256, 64, 0.1, P, fake, None) == 2
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3  # no workspace
+    o.causal = 0
+    V = lib.mxattn_forward_varlen
+    assert V(fake, fake, fake, fake, 0, 2, 100, 64, 0.1, P, fake, None) == 1     # nseq
+    assert V(fake, fake, fake, fake, 2, 2, 100, 96, 0.1, P, fake, None) == 1     # d
+    assert V(fake, fake, fake, None, 2, 2, 100, 64, 0.1, P, fake, None) == 1     # cu_seqlens
+    assert V(fake, fake, fake, fake, 2, 2, 100, 64, 0.1, P, fake, None) == 3     # no workspace
+    o.workspace, o.workspace_bytes = ctypes.c_void_p(0x100000), 1 << 30
+    assert V(fake, fake, fake, ctypes.c_void_p(0x1002), 2, 2, 100, 64, 0.1, P, fake, None) == 1  # unaligned
+    o.workspace, o.workspace_bytes = None, 0
     o.scale_rule = 3
     o.qmax = 9.0
     assert lib.mxattn_quant_v(fake, 1, 1, 256, 64, P, fake, fake, None) == 1

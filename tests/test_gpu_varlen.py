@@ -1,0 +1,153 @@
+"""Packed batches of variable-length sequences (mxattn_forward_varlen): token-major [T, H, d] inputs,
+device cu_seqlens.  Every sequence is an attention problem of its own, so the oracle runs each one
+alone (oracle.forward_varlen) and the comparison is element by element: rel-L2 <= 2e-3 over the
+batch, and per element max-abs <= 2e-2 in units of V ~ N(0, 1), widened for rows with a small row
+sum l to what one P^ code flip moves (see _flip_bound): short sequences have rows of a few keys,
+where one exp2 rounding that lands a P~ value on the other side of an E2M1 boundary is visible.
+Bit-exact checks tie the packing to the fixed-length kernels: every sequence equals mxattn_forward
+run on it alone, a single sequence equals mxattn_forward on [1, H, N, d], and equal-length
+sequences equal mxattn_forward with B = nseq."""
+import numpy as np
+import pytest
+
+import oracle
+from mxfp4_bit_attention_b200 import binding, inputs
+from helpers import MAX_ABS_TOL, REL_L2_TOL, out_to_numpy, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _draw(T, H, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H, d), dtype=np.float32)
+    k = rng.standard_normal((T, H, d), dtype=np.float32) * np.float32(1.5)
+    v = rng.standard_normal((T, H, d), dtype=np.float32)
+    if dtype == "bf16":
+        q, k, v = (inputs.bf16_bits_to_fp32(inputs.fp32_to_bf16_bits(x)) for x in (q, k, v))
+    return q, k, v
+
+
+def _dev(x, dtype):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def _cu(lengths):
+    import torch
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    return cu, torch.from_numpy(cu).cuda()
+
+
+def _check(got, ref, l=None, vmax=None):
+    assert np.isfinite(got).all()
+    e, m = rel_l2(got, ref), float(np.max(np.abs(got - ref)))
+    tol = MAX_ABS_TOL if l is None else _flip_bound(l, vmax)[:, :, None]
+    assert e <= REL_L2_TOL and bool(np.all(np.abs(got - ref) <= tol)), f"rel_l2={e:.3e} max_abs={m:.3e}"
+
+
+def _flip_bound(l, vmax):
+    """Per-row max-abs tolerance: 2e-2 plus what one P^ code flip can move.  P~ <= 1 puts every
+    group's scale at 2^-2 or below (UOS: the block max maps into (3.625, 7.25]), where neighbouring
+    E2M1 codes up to 4 are at most 1 apart: a flip moves one P^ value by <= 2^-2, hence the output
+    row sum(P^ V^) / l by <= 2^-2 (|V^| + |O|) / l <= 2 * 2^-2 * max|V^| / l (under PNQ l moves with
+    it).  max|V^| <= 4/3.625 max|V| (a block max scaled into (3.625, 7.25] rounds up to 4 at most)."""
+    return MAX_ABS_TOL + 0.5 * vmax / l
+
+
+@pytest.mark.parametrize("lengths,H,d,dtype", [
+    ([1], 1, 64, "fp32"),                        # one token
+    ([5, 0, 70, 1, 130], 2, 128, "bf16"),        # an empty sequence, ragged tails, one past a tile
+    ([128, 128, 64], 3, 64, "fp32"),             # whole tiles and a half tile
+    ([1000, 37, 300], 2, 128, "bf16"),           # several tiles per sequence
+    ([0, 0, 257], 1, 128, "bf16"),               # leading empty sequences
+])
+@pytest.mark.parametrize("pnq", [True, False])
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_matches_the_oracle(lengths, H, d, dtype, pnq, causal):
+    import torch
+    cu, cu_dev = _cu(lengths)
+    T = int(cu[-1])
+    q, k, v = _draw(T, H, d, dtype, seed=700 + T + d)
+    scale = float(np.float32(d ** -0.5))
+    opts = binding.Opts(pnq=pnq, causal=causal)
+    ws = torch.zeros(binding.load().mxattn_workspace_bytes_varlen(
+        len(lengths), H, T, d, binding.ctypes.byref(binding._copts(opts, binding._dtype_code(_dev(q[:1], dtype))))),
+        dtype=torch.uint8, device="cuda")
+    out = binding.mxattn_forward_varlen(_dev(q, dtype), _dev(k, dtype), _dev(v, dtype), cu_dev, scale, opts,
+                                        workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.mxattn_get_device_error(ws) == 0
+    ref, l = oracle.forward_varlen(q, k, v, cu, np.arange(T), scale, pnq=pnq, tau=8.0, causal=causal,
+                                   with_l=True)
+    ref = oracle.round_to_bf16(ref) if dtype == "bf16" else ref.astype(np.float32).astype(np.float64)
+    _check(out_to_numpy(out), ref, l, 4 / 3.625 * float(np.abs(v).max()))
+
+    # each sequence on its own through the fixed-length pass: the same bits
+    got = out.view(torch.int16 if dtype == "bf16" else torch.int32)
+    for s, n in enumerate(lengths):
+        if n == 0:
+            continue
+        lo = int(cu[s])
+        one = [x[lo:lo + n].transpose(0, 1).contiguous()[None] for x in (_dev(q, dtype), _dev(k, dtype), _dev(v, dtype))]
+        b = binding.mxattn_forward(*one, scale, opts)[0].transpose(0, 1).contiguous()
+        torch.cuda.synchronize()
+        assert torch.equal(got[lo:lo + n], b.view(got.dtype)), f"sequence {s} (length {n})"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_sequence_equals_the_fixed_length_pass(causal):
+    import torch
+    T, H, d = 1000, 4, 128
+    q, k, v = (_dev(x, "bf16") for x in _draw(T, H, d, "bf16", seed=5))
+    _, cu_dev = _cu([T])
+    opts = binding.Opts(causal=causal)
+    a = binding.mxattn_forward_varlen(q, k, v, cu_dev, 0.088, opts)
+    b = binding.mxattn_forward(*(x.transpose(0, 1).contiguous()[None] for x in (q, k, v)), 0.088, opts)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b[0].transpose(0, 1).contiguous().view(torch.int16))
+
+
+def test_equal_lengths_equal_the_batched_pass():
+    import torch
+    nseq, N, H, d = 3, 777, 2, 64
+    q, k, v = (_dev(x, "bf16") for x in _draw(nseq * N, H, d, "bf16", seed=6))
+    _, cu_dev = _cu([N] * nseq)
+    a = binding.mxattn_forward_varlen(q, k, v, cu_dev, 0.125)
+    bhnd = [x.view(nseq, N, H, d).transpose(1, 2).contiguous() for x in (q, k, v)]
+    b = binding.mxattn_forward(*bhnd, 0.125)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.transpose(1, 2).reshape(nseq * N, H, d).contiguous().view(torch.int16))
+
+
+def test_video_mix_sampled_rows():
+    """Three clips of different durations at 480p/720p-like token counts, 4 heads, sampled rows of
+    each sequence (first rows, tile edges, ragged tails) against the oracle."""
+    import torch
+    lengths = [32760, 4097, 20000]
+    cu, cu_dev = _cu(lengths)
+    T, H, d = int(cu[-1]), 4, 128
+    q, k, v = _draw(T, H, d, "bf16", seed=9)
+    out = binding.mxattn_forward_varlen(_dev(q, "bf16"), _dev(k, "bf16"), _dev(v, "bf16"), cu_dev, 0.088)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([cu[s] + inputs.sample_rows(n, 8) for s, n in enumerate(lengths)]))
+    ref = oracle.round_to_bf16(oracle.forward_varlen(q, k, v, cu, rows, 0.088, tau=8.0))
+    _check(out_to_numpy(out)[rows], ref)
+
+
+@pytest.mark.parametrize("table", [[0, 50, 40, 100], [0, 50, 100, 120], [3, 50, 80, 100]])
+def test_invalid_offsets_write_nothing_and_report(table):
+    """A cu_seqlens table that decreases, overshoots T or does not start at 0 is caught on the
+    device: the tile table is all zero, no later kernel writes, and the status reads as
+    MXATTN_ERR_INVALID_ARG."""
+    import torch
+    T, H, d = 100, 2, 64
+    q, k, v = (_dev(x, "fp32") for x in _draw(T, H, d, "fp32", seed=1))
+    cu_dev = torch.tensor(table, dtype=torch.int32, device="cuda")
+    opts = binding.Opts()
+    ws = torch.zeros(binding.load().mxattn_workspace_bytes_varlen(
+        3, H, T, d, binding.ctypes.byref(binding._copts(opts, binding.FP32))), dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, 7.0)
+    binding.mxattn_forward_varlen(q, k, v, cu_dev, 0.125, opts, out=out, workspace=ws)
+    assert binding.mxattn_get_device_error(ws) == 1
+    assert bool((out == 7.0).all())

@@ -145,3 +145,57 @@ def test_causal_first_row_sees_only_the_first_key(tiny):
     res = oracle.forward_rows(q[None], k[None], v[None], np.array([0]), 0.125, causal=True)["out"][0, 0]
     vq = oracle.prepare_head(q[:1], k, v)[2]
     np.testing.assert_array_equal(res, vq[0])
+
+
+def _packed(lengths, H, d, seed):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lengths))
+    q, k, v = (rng.standard_normal((T, H, d)).astype(np.float32) for _ in range(3))
+    return q, k, v, np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_quant_off_equals_block_diagonal_softmax(causal):
+    """A packed batch with quantization off is softmax attention over the whole packed token axis
+    with a block-diagonal mask (and the causal mask inside each block): built here densely."""
+    lengths = [5, 0, 70, 1, 130]
+    q, k, v, cu = _packed(lengths, 2, 64, seed=11)
+    T = len(q)
+    rows = np.arange(T)
+    s = 0.125
+    res = oracle.forward_varlen(q, k, v, cu, rows, s, quant=False, causal=causal)
+    seq = np.repeat(np.arange(len(lengths)), lengths)
+    for h in range(2):
+        qr = oracle.rotate_rows(q[:, h]).astype(np.float64)
+        kr = oracle.rotate_rows(k[:, h]).astype(np.float64)
+        S = (qr @ kr.T) * s
+        mask = seq[:, None] != seq[None, :]
+        if causal:
+            mask |= np.arange(T)[None, :] > np.arange(T)[:, None]
+        S[mask] = -np.inf
+        P = np.exp(S - S.max(axis=1, keepdims=True))
+        ref = (P / P.sum(axis=1, keepdims=True)) @ v[:, h].astype(np.float64)
+        np.testing.assert_allclose(res[:, h], ref, rtol=0, atol=1e-5)
+
+
+def test_varlen_sequences_are_independent():
+    """A sequence's output depends on its own tokens only: replacing every other sequence's Q, K and
+    V (whose V groups would share 32-key blocks with it if the groups ran across the packing) leaves
+    it unchanged bit for bit; packing the same tokens as one sequence does change it."""
+    lengths = [40, 100, 29]
+    q, k, v, cu = _packed(lengths, 1, 128, seed=12)
+    rows = np.arange(cu[1], cu[2])
+    a = oracle.forward_varlen(q, k, v, cu, rows, 0.09, tau=8.0)
+    rng = np.random.default_rng(99)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for x in (q2, k2, v2):
+        x[:cu[1]] = rng.standard_normal(x[:cu[1]].shape) * 7
+        x[cu[2]:] = rng.standard_normal(x[cu[2]:].shape) * 7
+    b = oracle.forward_varlen(q2, k2, v2, cu, rows, 0.09, tau=8.0)
+    np.testing.assert_array_equal(a, b)
+    whole = oracle.forward_varlen(q, k, v, np.array([0, len(q)]), rows, 0.09, tau=8.0)
+    assert np.abs(whole - a).max() > 1e-3
+    # one sequence of the whole batch is forward_rows on [H, T, d]
+    one = oracle.forward_rows(q.transpose(1, 0, 2).copy(), k.transpose(1, 0, 2).copy(),
+                              v.transpose(1, 0, 2).copy(), rows, 0.09, tau=8.0)["out"].transpose(1, 0, 2)
+    np.testing.assert_array_equal(whole, one)
