@@ -28,6 +28,7 @@ SRC = os.path.join(HERE, "mxref.c")
 LIB = os.path.join(HERE, "libmxref.so")
 
 RULE_UOS, RULE_QMAX6, RULE_OCP, RULE_CUSTOM = 0, 1, 2, 3
+FMT_MXFP4, FMT_NVFP4 = 0, 1   # 32-element groups with an E8M0 scale; 16-element blocks with an E4M3 scale
 RULES = {"uos": RULE_UOS, "qmax6": RULE_QMAX6, "ocp": RULE_OCP, "custom": RULE_CUSTOM}
 
 _lock = threading.Lock()
@@ -46,7 +47,7 @@ def build(force: bool = False) -> str:
 class AttnCfg(ctypes.Structure):
     _fields_ = [("key_tile", ctypes.c_int), ("pnq", ctypes.c_int), ("quant_p", ctypes.c_int),
                 ("rule", ctypes.c_int), ("qmax", ctypes.c_double), ("tau", ctypes.c_double),
-                ("qpos", ctypes.c_void_p)]
+                ("qpos", ctypes.c_void_p), ("fmt", ctypes.c_int)]
 
 
 def lib():
@@ -78,6 +79,16 @@ def lib():
             L.mxref_attention_rows.restype = None
             L.mxref_qmax_sweep.argtypes = [P, i64, i64, i32, P, i32, P, P]
             L.mxref_qmax_sweep.restype = None
+            L.mxref_e4m3_decode.argtypes = [i32]
+            L.mxref_e4m3_decode.restype = f64
+            L.mxref_e4m3_encode.argtypes = [f64]
+            L.mxref_e4m3_encode.restype = i32
+            L.mxref_quantize_nvfp4.argtypes = [P, i64, i64, i32, P, P]
+            L.mxref_quantize_nvfp4.restype = None
+            L.mxref_dequantize_nvfp4.argtypes = [P, P, i64, P]
+            L.mxref_dequantize_nvfp4.restype = None
+            L.mxref_rotate_quantize_rows_nvfp4.argtypes = [P, i64, i32, i32, P, P]
+            L.mxref_rotate_quantize_rows_nvfp4.restype = None
             L.mxref_num_threads.argtypes = []
             L.mxref_num_threads.restype = i32
             _lib = L
@@ -108,21 +119,39 @@ def scale_exponent(amax: float, rule: int = RULE_UOS, qmax: float = 7.25) -> int
     return int(lib().mxref_scale_exponent(float(amax), int(rule), float(qmax)))
 
 
+def e4m3_encode(v: float) -> int:
+    """E4M3 byte nearest to v (ties to even, saturating at 448): the NVFP4 block scale."""
+    return int(lib().mxref_e4m3_encode(float(v)))
+
+
+def e4m3_decode(byte: int) -> float:
+    return float(lib().mxref_e4m3_decode(int(byte)))
+
+
+def block_size(fmt: int) -> int:
+    return 16 if fmt == FMT_NVFP4 else 32
+
+
 # ----------------------------------------------------------------------------------------------
 # Quantization
 # ----------------------------------------------------------------------------------------------
 
-def quantize(x: np.ndarray, axis: int = 0, rule: int = RULE_UOS, qmax: float = 7.25):
+def quantize(x: np.ndarray, axis: int = 0, rule: int = RULE_UOS, qmax: float = 7.25, fmt: int = FMT_MXFP4):
     """MXFP4-quantize a 2-D fp32 matrix in groups of 32 along columns (axis 0)
     or along rows (axis 1, output transposed).  Returns (codes, scales) with
-    codes unpacked, one 4-bit code per byte: [outer, ceil(inner/32)*32]."""
+    codes unpacked, one 4-bit code per byte: [outer, ceil(inner/32)*32].
+    fmt = FMT_NVFP4: blocks of 16 with E4M3 scale bytes (rule and qmax unused)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     rows, cols = x.shape
     outer, inner = (rows, cols) if axis == 0 else (cols, rows)
-    ng = (inner + 31) // 32
-    codes = np.zeros((outer, ng * 32), np.uint8)
+    bs = block_size(fmt)
+    ng = (inner + bs - 1) // bs
+    codes = np.zeros((outer, ng * bs), np.uint8)
     scales = np.zeros((outer, ng), np.uint8)
-    lib().mxref_quantize(_ptr(x), rows, cols, axis, rule, qmax, _ptr(codes), _ptr(scales))
+    if fmt == FMT_NVFP4:
+        lib().mxref_quantize_nvfp4(_ptr(x), rows, cols, axis, _ptr(codes), _ptr(scales))
+    else:
+        lib().mxref_quantize(_ptr(x), rows, cols, axis, rule, qmax, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
@@ -134,27 +163,34 @@ def rotate_rows(x: np.ndarray) -> np.ndarray:
     return y
 
 
-def rotate_quantize_rows(x: np.ndarray, rotate: bool = True, rule: int = RULE_UOS, qmax: float = 7.25):
-    """Q/K operand: optional rotation then groups of 32 along d.
-    Returns unpacked codes [rows, d] and scales [rows, d/32]."""
+def rotate_quantize_rows(x: np.ndarray, rotate: bool = True, rule: int = RULE_UOS, qmax: float = 7.25,
+                         fmt: int = FMT_MXFP4):
+    """Q/K operand: optional rotation then groups of 32 along d (NVFP4: blocks of 16).
+    Returns unpacked codes [rows, d] and scales [rows, d/32] (NVFP4: [rows, d/16])."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     d = x.shape[-1]
     x2 = x.reshape(-1, d)
     rows = x2.shape[0]
     codes = np.zeros((rows, d), np.uint8)
-    scales = np.zeros((rows, d // 32), np.uint8)
-    lib().mxref_rotate_quantize_rows(_ptr(x2), rows, d, int(bool(rotate)), rule, qmax, _ptr(codes),
-                                     _ptr(scales))
+    scales = np.zeros((rows, d // block_size(fmt)), np.uint8)
+    if fmt == FMT_NVFP4:
+        lib().mxref_rotate_quantize_rows_nvfp4(_ptr(x2), rows, d, int(bool(rotate)), _ptr(codes), _ptr(scales))
+    else:
+        lib().mxref_rotate_quantize_rows(_ptr(x2), rows, d, int(bool(rotate)), rule, qmax, _ptr(codes),
+                                         _ptr(scales))
     return codes, scales
 
 
-def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
-    """Exact values of unpacked codes with one scale byte per 32 codes (fp64)."""
+def dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int = FMT_MXFP4) -> np.ndarray:
+    """Exact values of unpacked codes with one scale byte per 32 codes (NVFP4: per 16) (fp64)."""
     codes = np.ascontiguousarray(codes, dtype=np.uint8)
     scales = np.ascontiguousarray(scales, dtype=np.uint8)
-    assert codes.size == scales.size * 32
+    assert codes.size == scales.size * block_size(fmt)
     out = np.empty(codes.shape, np.float64)
-    lib().mxref_dequantize(_ptr(codes), _ptr(scales), scales.size, _ptr(out))
+    if fmt == FMT_NVFP4:
+        lib().mxref_dequantize_nvfp4(_ptr(codes), _ptr(scales), scales.size, _ptr(out))
+    else:
+        lib().mxref_dequantize(_ptr(codes), _ptr(scales), scales.size, _ptr(out))
     return out
 
 
@@ -163,11 +199,12 @@ def dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------------------------
 
 def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=True, rule=RULE_UOS,
-                   qmax=7.25, tau=0.0, weights=False, codes=False, qpos=None):
+                   qmax=7.25, tau=0.0, weights=False, codes=False, qpos=None, fmt=FMT_MXFP4):
     """Online-softmax attention with PNQ for query rows qd [n, d] against
     kd, vd [N, d] (fp64 values).  Returns dict(out, m, l[, wsum, ocheck]
     [, p_codes [n, ntiles*key_tile], p_scales [n, ntiles*key_tile/32]]).  qpos: causal masking,
-    row i sees keys 0..qpos[i] (None: all keys)."""
+    row i sees keys 0..qpos[i] (None: all keys).  fmt = FMT_NVFP4: P~ in NVFP4 blocks of 16
+    (p_scales [n, ntiles*key_tile/16], E4M3 bytes)."""
     qd = np.ascontiguousarray(qd, dtype=np.float64)
     kd = np.ascontiguousarray(kd, dtype=np.float64)
     vd = np.ascontiguousarray(vd, dtype=np.float64)
@@ -176,7 +213,7 @@ def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=Tru
     assert kd.shape == (N, d) and vd.shape == (N, d) and key_tile % 32 == 0
     qp = None if qpos is None else np.ascontiguousarray(qpos, dtype=np.int64)
     cfg = AttnCfg(int(key_tile), int(bool(pnq)), int(bool(quant_p)), int(rule), float(qmax), float(tau),
-                  None if qp is None else qp.ctypes.data)
+                  None if qp is None else qp.ctypes.data, int(fmt))
     out = np.empty((n, d), np.float64)
     m = np.empty(n, np.float64)
     l = np.empty(n, np.float64)
@@ -184,7 +221,7 @@ def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=Tru
     ocheck = np.empty((n, d), np.float64) if weights else None
     ntiles = (N + key_tile - 1) // key_tile
     pc = np.zeros((n, ntiles * key_tile), np.uint8) if codes else None
-    ps = np.zeros((n, ntiles * key_tile // 32), np.uint8) if codes else None
+    ps = np.zeros((n, ntiles * key_tile // block_size(fmt)), np.uint8) if codes else None
     lib().mxref_attention_rows(_ptr(qd), n, _ptr(kd), _ptr(vd), N, d, float(np.float32(softmax_scale)),
                                ctypes.byref(cfg), _ptr(out), _ptr(m), _ptr(l), _ptr(wsum), _ptr(ocheck),
                                _ptr(pc), _ptr(ps))
@@ -198,10 +235,10 @@ def attention_rows(qd, kd, vd, softmax_scale, key_tile=64, pnq=True, quant_p=Tru
     return res
 
 
-def prepare_head(q, k, v, rotate=True, rule=RULE_UOS, qmax=7.25, quant=True):
+def prepare_head(q, k, v, rotate=True, rule=RULE_UOS, qmax=7.25, quant=True, fmt=FMT_MXFP4):
     """Rotate/quantize one head's Q [nq, d], K [N, d], V [N, d] (fp32) and
     return their exact dequantized values (fp64): Q, K groups along d, V
-    groups of 32 consecutive keys per channel."""
+    groups of 32 consecutive keys per channel (NVFP4: blocks of 16)."""
     q = np.ascontiguousarray(q, dtype=np.float32)
     k = np.ascontiguousarray(k, dtype=np.float32)
     v = np.ascontiguousarray(v, dtype=np.float32)
@@ -209,30 +246,31 @@ def prepare_head(q, k, v, rotate=True, rule=RULE_UOS, qmax=7.25, quant=True):
         qr = rotate_rows(q) if rotate else q
         kr = rotate_rows(k) if rotate else k
         return qr.astype(np.float64), kr.astype(np.float64), v.astype(np.float64)
-    qc, qs = rotate_quantize_rows(q, rotate, rule, qmax)
-    kc, ks = rotate_quantize_rows(k, rotate, rule, qmax)
-    vc, vs = quantize(v, axis=1, rule=rule, qmax=qmax)      # [d, ceil(N/32)*32]
+    qc, qs = rotate_quantize_rows(q, rotate, rule, qmax, fmt)
+    kc, ks = rotate_quantize_rows(k, rotate, rule, qmax, fmt)
+    vc, vs = quantize(v, axis=1, rule=rule, qmax=qmax, fmt=fmt)  # [d, ceil(N/bs)*bs]
     N = v.shape[0]
-    vd = dequantize(vc, vs)[:, :N].T                           # [N, d]
-    return dequantize(qc, qs), dequantize(kc, ks), np.ascontiguousarray(vd)
+    vd = dequantize(vc, vs, fmt)[:, :N].T                           # [N, d]
+    return dequantize(qc, qs, fmt), dequantize(kc, ks, fmt), np.ascontiguousarray(vd)
 
 
 def forward_rows(q, k, v, rows, softmax_scale, rotate=True, rule=RULE_UOS, qmax=7.25, pnq=True,
-                 key_tile=64, tau=0.0, quant=True, weights=False, causal=False):
+                 key_tile=64, tau=0.0, quant=True, weights=False, causal=False, fmt=FMT_MXFP4):
     """MXAttention forward for selected query rows of every head.
 
     q, k, v: fp32 arrays [BH, N, d] (exact upcasts of the inputs).
     rows:    int array of query indices (same rows for every head).
     causal:  each row sees only the keys up to its own index (self-attention, top-left aligned).
+    fmt:     FMT_MXFP4 (the method) or FMT_NVFP4 (the comparison format) for Q, K, V and P~.
     Returns dict with out [BH, len(rows), d] (fp64) and m, l [BH, len(rows)].
     """
     BH, N, d = q.shape
     rows = np.asarray(rows, dtype=np.int64)
     outs, ms, ls, ws, ocs = [], [], [], [], []
     for h in range(BH):
-        qd, kd, vd = prepare_head(q[h][rows], k[h], v[h], rotate, rule, qmax, quant)
+        qd, kd, vd = prepare_head(q[h][rows], k[h], v[h], rotate, rule, qmax, quant, fmt)
         r = attention_rows(qd, kd, vd, softmax_scale, key_tile, pnq, quant, rule, qmax, tau, weights,
-                           qpos=rows if causal else None)
+                           qpos=rows if causal else None, fmt=fmt)
         outs.append(r["out"])
         ms.append(r["m"])
         ls.append(r["l"])

@@ -134,6 +134,96 @@ static int quantize_group(const float* x, int64_t n, int64_t stride, int rule, d
 }
 
 /*
+ * NVFP4 comparison format (the pages compare MXAttention against NVFP4-based
+ * baselines without defining the format; this is the public NVFP4 layout as
+ * read for that comparison): blocks of 16 E2M1 codes sharing one scale that is
+ * an FP8 E4M3 number (sign 0, 4 exponent bits with bias 7, 3 mantissa bits,
+ * subnormals down to 2^-9, largest finite 448; the two NaN bytes 0x7F/0xFF are
+ * never produced).
+ */
+
+/* Value of an E4M3 byte (bit 7 = sign; 0x7F/0xFF = NaN). */
+double mxref_e4m3_decode(int byte) {
+  int mag = byte & 0x7F;
+  if (mag == 0x7F) return NAN;
+  int e = mag >> 3, m = mag & 7;
+  double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return (byte & 0x80) ? -v : v;
+}
+
+/*
+ * Round v to the nearest E4M3 value, ties to the even byte (mantissa bit 0
+ * clear), magnitudes above 448 saturating to 448 (the "satfinite" mode).
+ * Searched over all 127 finite magnitudes.
+ */
+int mxref_e4m3_encode(double v) {
+  int sign = signbit(v) ? 0x80 : 0;
+  double a = fabs(v);
+  int best = 0;
+  double best_d = a;
+  for (int b = 1; b < 0x7F; b++) {
+    double dist = fabs(a - mxref_e4m3_decode(b));
+    if (dist < best_d || (dist == best_d && (b & 1) == 0)) {
+      best = b;
+      best_d = dist;
+    }
+  }
+  if (a >= 448.0) best = 0x7E;
+  return sign | best;
+}
+
+/*
+ * One NVFP4 block of n (<= 16) values read with a stride (missing members are
+ * zeros).  Readings: the scale is the E4M3 rounding of fl32(amax / 6) (the block
+ * maximum lands on the largest code, 6, up to the scale's rounding); each value
+ * is divided by the scale in fp32 (one IEEE rounding) and rounded to E2M1 with
+ * saturation; a scale that rounds to 0 gives all-zero codes.  Returns the scale
+ * byte.
+ */
+static int quantize_block16(const float* x, int64_t n, int64_t stride, uint8_t* codes) {
+  float amax = 0.0f;
+  for (int64_t i = 0; i < n; i++) {
+    float a = fabsf(x[i * stride]);
+    if (a > amax) amax = a;
+  }
+  int sb = mxref_e4m3_encode((double)(amax / 6.0f));
+  float s = (float)mxref_e4m3_decode(sb);
+  for (int64_t i = 0; i < n; i++) codes[i] = s > 0.0f ? (uint8_t)mxref_e2m1_encode((double)(x[i * stride] / s)) : 0;
+  return sb;
+}
+
+/*
+ * NVFP4 quantization of a row-major [rows][cols] fp32 matrix, the layout of
+ * mxref_quantize with blocks of 16: axis 0 along a row (codes [rows][ceil(cols/16)*16],
+ * scales [rows][ceil(cols/16)]), axis 1 along a column (output transposed).
+ */
+void mxref_quantize_nvfp4(const float* x, int64_t rows, int64_t cols, int axis, uint8_t* codes, uint8_t* scales) {
+  int64_t outer = axis == 0 ? rows : cols;
+  int64_t inner = axis == 0 ? cols : rows;
+  int64_t nb = (inner + 15) / 16;
+#pragma omp parallel for schedule(static)
+  for (int64_t o = 0; o < outer; o++) {
+    for (int64_t b = 0; b < nb; b++) {
+      int64_t i0 = b * 16;
+      int64_t n = inner - i0 < 16 ? inner - i0 : 16;
+      const float* base = axis == 0 ? x + o * cols + i0 : x + i0 * cols + o;
+      uint8_t* c = codes + o * nb * 16 + i0;
+      memset(c, 0, 16);
+      scales[o * nb + b] = (uint8_t)quantize_block16(base, n, axis == 0 ? 1 : cols, c);
+    }
+  }
+}
+
+/* Dequantize unpacked NVFP4 codes: out[i] = decode(code) * e4m3(scale of its block of 16). */
+void mxref_dequantize_nvfp4(const uint8_t* codes, const uint8_t* scales, int64_t nblocks, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t b = 0; b < nblocks; b++) {
+    double s = mxref_e4m3_decode(scales[b]);
+    for (int i = 0; i < 16; i++) out[b * 16 + i] = mxref_e2m1_decode(codes[b * 16 + i]) * s;
+  }
+}
+
+/*
  * Generic MXFP4 quantization of a row-major [rows][cols] fp32 matrix.
  *  axis 0: groups of 32 consecutive columns within a row.
  *     codes  [rows][ceil(cols/32)*32] one code per byte (unpacked)
@@ -206,6 +296,19 @@ void mxref_rotate_quantize_rows(const float* x, int64_t rows, int d, int rotate,
   }
 }
 
+/* The same with NVFP4 blocks of 16 along d: codes [rows][d], scales [rows][d/16]. */
+void mxref_rotate_quantize_rows_nvfp4(const float* x, int64_t rows, int d, int rotate, uint8_t* codes,
+                                      uint8_t* scales) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; r++) {
+    float buf[1024];
+    memcpy(buf, x + r * d, sizeof(float) * (size_t)d);
+    if (rotate) mxref_fwht_row(buf, d);
+    for (int b = 0; b < d / 16; b++)
+      scales[r * (d / 16) + b] = (uint8_t)quantize_block16(buf + b * 16, 16, 1, codes + r * d + b * 16);
+  }
+}
+
 /* Rotation alone (for the rotation-only and quantization-off checks). */
 void mxref_rotate_rows(float* x, int64_t rows, int d) {
 #pragma omp parallel for schedule(static)
@@ -230,7 +333,15 @@ typedef struct {
   double tau;     /* lazy max update threshold in log2 units; 0 = eager      */
   const int64_t* qpos; /* causal masking: key k is seen by row r only if k <= qpos[r]
                           (the row's position in the sequence); NULL: every key     */
+  int fmt;        /* 0: MXFP4 (groups of 32, E8M0 scale by `rule`);
+                     1: NVFP4 (blocks of 16, E4M3 scale), see below              */
 } mxref_attn_cfg;
+
+/* NVFP4 exponential tiles: P~ <= 1 is first multiplied by this tensor-level factor, 448 * 6, so
+   that the block holding the running max (P~ = 1) gets the largest E4M3 scale, 448, and its
+   maximum the largest code, 6; smaller blocks keep the E4M3 scale's full range.  P^ is divided
+   by it again (it cancels in O = O~ / l either way). */
+#define MXREF_NVFP4_P_GLOBAL 2688.0f
 
 /*
  * Online-softmax attention for a set of query rows of one head, following the
@@ -248,7 +359,9 @@ typedef struct {
  *   alpha = exp(m_old - m_new)             (unquantized)
  *   P~_k  = fl32(exp(x_k - m_new))  for keys < N, 0 beyond N
  *   P^    = MXFP4(P~) in groups of 32 keys from the tile start, same rule as
- *           Q/K/V (Fig. 1: UOS applies to all quantized attention tensors)
+ *           Q/K/V (Fig. 1: UOS applies to all quantized attention tensors);
+ *           with fmt = 1, NVFP4 blocks of 16 keys of fl32(P~ * 2688), divided
+ *           by 2688 again
  *   l     = alpha*l + sum P^   (PNQ)   or   alpha*l + sum P~   (direct)
  *   O~    = alpha*O~ + sum_k P^_k v_k
  * O = O~ / l.
@@ -259,7 +372,8 @@ typedef struct {
  * the output rebuilt from those weights (both need wsum and ocheck non-NULL).
  * pcodes [nrows][ntiles*T] and pscales [nrows][ntiles*T/32], when non-NULL,
  * receive the E2M1 codes (one per byte, keys in order, padded keys 0) and the
- * E8M0 scale bytes of every quantized P~ group (quant_p only).
+ * E8M0 scale bytes of every quantized P~ group (quant_p only; NVFP4: the E4M3
+ * bytes of the blocks of 16, [nrows][ntiles*T/16]).
  */
 void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const double* v, int N,
                           int d, float scale, const mxref_attn_cfg* cfg, double* out, double* m_out,
@@ -303,7 +417,18 @@ void mxref_attention_rows(const double* q, int64_t nrows, const double* k, const
         double alpha = (m == -INFINITY) ? 0.0 : exp((double)m - (double)mnew);
         m = mnew;
         for (int j = 0; j < T; j++) pt[j] = j < nk ? (float)exp((double)x[j] - (double)m) : 0.0f;
-        if (cfg->quant_p) {
+        if (cfg->quant_p && cfg->fmt == 1) {
+          for (int b = 0; b < T / 16; b++) {
+            float y[16];
+            for (int i = 0; i < 16; i++) y[i] = pt[b * 16 + i] * MXREF_NVFP4_P_GLOBAL;
+            int sb = quantize_block16(y, 16, 1, codes);
+            double sv = mxref_e4m3_decode(sb);
+            for (int i = 0; i < 16; i++)
+              ph[b * 16 + i] = mxref_e2m1_decode(codes[i]) * sv / (double)MXREF_NVFP4_P_GLOBAL;
+            if (pcodes_out) memcpy(pcodes_out + ((size_t)r * ntiles + t) * T + b * 16, codes, 16);
+            if (pscales_out) pscales_out[((size_t)r * ntiles + t) * (T / 16) + b] = (uint8_t)sb;
+          }
+        } else if (cfg->quant_p) {
           for (int g = 0; g < T / 32; g++) {
             int sb = quantize_group(pt + g * 32, 32, 1, cfg->rule, cfg->qmax, codes);
             for (int i = 0; i < 32; i++) ph[g * 32 + i] = ldexp(mxref_e2m1_decode(codes[i]), sb - 127);
