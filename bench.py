@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4"],
+                    help="element format: the method's MXFP4, or the NVFP4 comparison format")
     ap.add_argument("--causal", action="store_true",
                     help="causal self-attention; TFLOPS count the visible (query, key) pairs, N(N+1)/2 per head")
     return ap.parse_args()
@@ -284,11 +286,12 @@ def main():
     hq, hk, hv = (host_tensor(g[n]) for n in "qkv")
     del g
     q, k, v = (t.to(dev) for t in (hq, hk, hv))
-    opts = binding.Opts(causal=args.causal)
+    opts = binding.Opts(causal=args.causal,
+                        format=binding.FMT_NVFP4 if args.format == "nvfp4" else binding.FMT_MXFP4)
     scale = float(np.float32(w.d ** -0.5))
     ws = binding.new_workspace(1, w.H, w.N, w.d, opts, dev)
     out = torch.empty(shape, dtype=tdt, device=dev)
-    sizes = binding.operand_sizes(1, w.H, w.N, w.d)
+    sizes = binding.operand_sizes(1, w.H, w.N, w.d, opts.format)
     # the packed operands live inside the workspace; carve the same views for the split calls
     ops = {}
     off = 256
@@ -380,8 +383,9 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "fp4(e2m1)+fp32 accumulate, bf16 in/out", "data": "synthetic",
                 "config": {"workload": w.name, "B": world, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
-                           "key_tile": 64, "scale_rule": "UOS Qmax=7.25", "pnq": True, "rotate": True,
-                           "causal": args.causal,
+                           "key_tile": 64, "pnq": True, "rotate": True, "causal": args.causal,
+                           "format": args.format,
+                           "scale_rule": "UOS Qmax=7.25" if args.format == "mxfp4" else "E4M3(amax/6) per 16",
                            "rescale_tau": opts.rescale_tau, "parallelism": f"independent problems x{world}",
                            "l2": "inputs (2.3 GB) larger than L2 (126 MB); no flush"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,

@@ -61,6 +61,21 @@
  *             the scale of channel c, key group g (0..3) at byte
  *             (c % 32)*16 + (c / 32)*4 + g.  Channels >= d are zero.
  *
+ * NVFP4 comparison format (opts->format = MXATTN_FMT_NVFP4): the same codes,
+ * in blocks of 16 elements whose scales are E4M3 bytes (FP8: bias 7, 3
+ * mantissa bits, subnormals, largest 448; scale = E4M3(fl32(amax / 6)), codes
+ * of fl32(x / scale), a zero scale gives zero codes).  The scale atoms hold
+ * 4 blocks (64 elements) per row:
+ *  QK scales  [B*H][T128][d/64][512]: atom a covers dims 64a .. 64a+63, block
+ *             b (0..3) of token r at byte (r % 32)*16 + (r / 32)*4 + b.
+ *  V scales   [B*H][T64][512]: one atom per 64-key tile, key block b (0..3)
+ *             of channel c at byte (c % 32)*16 + (c / 32)*4 + b.
+ * The pages compare MXAttention with NVFP4-based baselines without defining
+ * NVFP4; this is the public format, built for that comparison (full attention,
+ * no dump, no causal or varlen).  The exponential tile P~ <= 1 is scaled by
+ * 448*6 before its blocks take their scales (the block holding the running
+ * max gets scale 448); the factor cancels in O = O~/l.
+ *
  * Workspace (mxattn_forward, mxattn_attention_mxfp4): opts->workspace is a
  * device buffer of at least mxattn_workspace_bytes() bytes, 256-byte aligned.
  * Its first 256 bytes are a status block that the kernels set when a bounded
@@ -103,6 +118,11 @@ typedef enum mxattn_scale_rule {
 
 typedef enum mxattn_dtype { MXATTN_BF16 = 0, MXATTN_FP32 = 1 } mxattn_dtype;
 
+typedef enum mxattn_format {
+  MXATTN_FMT_MXFP4 = 0,  /* 32-element groups, E8M0 scale chosen by opts.scale_rule */
+  MXATTN_FMT_NVFP4 = 1   /* 16-element blocks, E4M3 scale (comparison format)       */
+} mxattn_format;
+
 typedef struct mxattn_opts {
   int scale_rule;          /* mxattn_scale_rule, used for Q, K, V and the P~ tiles      */
   float qmax;              /* boundary for MXATTN_SCALE_CEIL_CUSTOM                      */
@@ -126,18 +146,22 @@ typedef struct mxattn_opts {
                            /* ways and fix none); key tiles past a query tile's diagonal */
                            /* are skipped.  Self-attention entry points only (varlen:    */
                            /* within each sequence); cross-attention returns             */
-                           /* MXATTN_ERR_UNSUPPORTED.  0 = full attention.               */
+                           /* MXATTN_ERR_UNSUPPORTED, as does NVFP4.  0 = full attention. */
+  int format;              /* mxattn_format: MXFP4 (the method) or NVFP4 (comparison)     */
 } mxattn_opts;
 
 /* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
- * key_tile 64, rescale_tau 8, no workspace, default wait budget, causal 0. */
+ * key_tile 64, rescale_tau 8, no workspace, default wait budget, MXFP4,
+ * causal 0. */
 MXATTN_API void mxattn_opts_default(mxattn_opts* opts);
 
 /* Bytes of workspace mxattn_forward needs for this problem (status block plus
  * packed Q, K, V operands); 0 for invalid sizes. */
 MXATTN_API size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts);
 
-/* Sizes of the packed attention operands described above (0 for invalid sizes). */
+/* Sizes of the packed attention operands described above (0 for invalid sizes),
+ * MXFP4; NVFP4 needs d/64 times the QK scale bytes and ceil(N/64)*512 per head
+ * for the V scales (mxattn_workspace_bytes takes the format from opts). */
 MXATTN_API size_t mxattn_qk_codes_bytes(int B, int H, int N, int d);
 MXATTN_API size_t mxattn_qk_scales_bytes(int B, int H, int N, int d);
 MXATTN_API size_t mxattn_v_codes_bytes(int B, int H, int N, int d);
@@ -156,6 +180,8 @@ MXATTN_API mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* st
  *                transposed: codes [cols][ceil(rows/32)*16],
  *                scales [cols][ceil(rows/32)].
  * Partial tail groups are zero-padded.  No rotation is applied.
+ * opts->format = MXATTN_FMT_NVFP4: blocks of 16 with E4M3 scale bytes
+ * (codes [outer][ceil(inner/16)*8], scales [outer][ceil(inner/16)]).
  */
 MXATTN_API mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, int group_axis,
                                     const mxattn_opts* opts, uint8_t* codes, uint8_t* scales,

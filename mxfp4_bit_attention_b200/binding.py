@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 
 SCALE_UOS, SCALE_QMAX6, SCALE_OCP, SCALE_CEIL_CUSTOM = 0, 1, 2, 3
 BF16, FP32 = 0, 1
+FMT_MXFP4, FMT_NVFP4 = 0, 1
 
 STATUS = {0: "MXATTN_OK", 1: "MXATTN_ERR_INVALID_ARG", 2: "MXATTN_ERR_UNSUPPORTED",
           3: "MXATTN_ERR_WORKSPACE", 4: "MXATTN_ERR_CUDA", 5: "MXATTN_ERR_TIMEOUT"}
@@ -42,7 +43,7 @@ class COpts(ctypes.Structure):
                 ("rotate", ctypes.c_int), ("dtype", ctypes.c_int), ("key_tile", ctypes.c_int),
                 ("rescale_tau", ctypes.c_float), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("wait_budget_cycles", ctypes.c_longlong),
-                ("causal", ctypes.c_int)]
+                ("causal", ctypes.c_int), ("format", ctypes.c_int)]
 
 
 @dataclass
@@ -55,6 +56,7 @@ class Opts:
     rescale_tau: float = 8.0
     wait_budget_cycles: int = 0  # 0: the library's default (about one second)
     causal: bool = False  # self-attention: query row i sees keys 0..i
+    format: int = 0       # FMT_MXFP4 (the method) or FMT_NVFP4 (the comparison format)
 
 
 def lib_path() -> str:
@@ -138,6 +140,7 @@ def _copts(o: Opts | None, dtype: int, workspace=None) -> COpts:
     c.dtype, c.key_tile, c.rescale_tau = dtype, int(o.key_tile), float(o.rescale_tau)
     c.wait_budget_cycles = int(o.wait_budget_cycles)
     c.causal = int(bool(o.causal))
+    c.format = int(o.format)
     if workspace is not None:
         c.workspace = ctypes.c_void_p(workspace.data_ptr())
         c.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -148,11 +151,17 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def operand_sizes(B: int, H: int, N: int, d: int) -> dict:
+def operand_sizes(B: int, H: int, N: int, d: int, fmt: int = FMT_MXFP4) -> dict:
+    """Bytes of the packed operands; NVFP4 scales per the header (d/64 Q/K atoms per 128-row tile,
+    one V atom per 64-key tile)."""
     L = load()
-    return {"q_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "q_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
-            "k_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "k_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
-            "v_codes": L.mxattn_v_codes_bytes(B, H, N, d), "v_scales": L.mxattn_v_scales_bytes(B, H, N, d)}
+    s = {"q_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "q_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
+         "k_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "k_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
+         "v_codes": L.mxattn_v_codes_bytes(B, H, N, d), "v_scales": L.mxattn_v_scales_bytes(B, H, N, d)}
+    if fmt == FMT_NVFP4:
+        s["q_scales"] = s["k_scales"] = s["q_scales"] * (d // 64)
+        s["v_scales"] = B * H * ((N + 63) // 64) * 512
+    return s
 
 
 def mxattn_workspace_bytes(B: int, H: int, N: int, d: int, opts: Opts | None = None) -> int:
@@ -171,8 +180,9 @@ def mxattn_quantize_mxfp4(x, group_axis=0, opts: Opts | None = None, codes=None,
     import torch
     rows, cols = x.shape
     outer, inner = (rows, cols) if group_axis == 0 else (cols, rows)
-    ng = (inner + 31) // 32
-    codes = codes if codes is not None else torch.empty((outer, ng * 16), dtype=torch.uint8, device=x.device)
+    gs = 16 if (opts is not None and opts.format == FMT_NVFP4) else 32
+    ng = (inner + gs - 1) // gs
+    codes = codes if codes is not None else torch.empty((outer, ng * gs // 2), dtype=torch.uint8, device=x.device)
     scales = scales if scales is not None else torch.empty((outer, ng), dtype=torch.uint8, device=x.device)
     c = _copts(opts, _dtype_code(x))
     _check("mxattn_quantize_mxfp4", load().mxattn_quantize_mxfp4(
@@ -180,16 +190,16 @@ def mxattn_quantize_mxfp4(x, group_axis=0, opts: Opts | None = None, codes=None,
     return codes, scales
 
 
-def _alloc_operands(B, H, N, d, device):
+def _alloc_operands(B, H, N, d, device, fmt=FMT_MXFP4):
     import torch
-    s = operand_sizes(B, H, N, d)
+    s = operand_sizes(B, H, N, d, fmt)
     return {k: torch.empty(v, dtype=torch.uint8, device=device) for k, v in s.items()}
 
 
 def mxattn_hadamard_quant_qk(q, k, opts: Opts | None = None, out=None, stream=None):
     """Rotate + quantize Q and K ([B, H, N, d]) into the packed QK operand layout."""
     B, H, N, d = q.shape
-    out = out or _alloc_operands(B, H, N, d, q.device)
+    out = out or _alloc_operands(B, H, N, d, q.device, (opts or Opts()).format)
     c = _copts(opts, _dtype_code(q))
     _check("mxattn_hadamard_quant_qk", load().mxattn_hadamard_quant_qk(
         _ptr(q), _ptr(k), B, H, N, d, ctypes.byref(c), _ptr(out["q_codes"]), _ptr(out["q_scales"]),
@@ -200,7 +210,7 @@ def mxattn_hadamard_quant_qk(q, k, opts: Opts | None = None, out=None, stream=No
 def mxattn_quant_v(v, opts: Opts | None = None, out=None, stream=None):
     """Quantize V ([B, H, N, d]) along keys into the packed V operand layout."""
     B, H, N, d = v.shape
-    out = out or _alloc_operands(B, H, N, d, v.device)
+    out = out or _alloc_operands(B, H, N, d, v.device, (opts or Opts()).format)
     c = _copts(opts, _dtype_code(v))
     _check("mxattn_quant_v", load().mxattn_quant_v(
         _ptr(v), B, H, N, d, ctypes.byref(c), _ptr(out["v_codes"]), _ptr(out["v_scales"]), _stream(stream)))

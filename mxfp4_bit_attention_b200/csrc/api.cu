@@ -28,6 +28,15 @@ bool sizes_ok(int B, int H, int N, int d) {
 int64_t t128(int N) { return ((int64_t)N + 127) / 128; }
 int64_t t64(int N) { return ((int64_t)N + 63) / 64; }
 
+// Scale bytes of the packed operands: MXFP4 one 512-byte atom per 128-row Q/K tile and per
+// 128-key V tile; NVFP4 (16-element blocks) d/64 atoms per Q/K tile and one per 64-key V tile.
+size_t qk_scale_bytes(int B, int H, int N, int d, int fmt) {
+  return (size_t)B * H * t128(N) * 512 * (fmt == MXATTN_FMT_NVFP4 ? d / 64 : 1);
+}
+size_t v_scale_bytes(int B, int H, int N, int fmt) {
+  return (size_t)B * H * (fmt == MXATTN_FMT_NVFP4 ? t64(N) : t128(N)) * 512;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Boundary q = mq * 2^eq of a ceiling rule, or the OCP floor rule.
@@ -62,6 +71,8 @@ mxattn_status check_opts(const mxattn_opts* o) {
   if (o->key_tile != 64) return o->key_tile == 128 ? MXATTN_ERR_UNSUPPORTED : MXATTN_ERR_INVALID_ARG;
   if (o->wait_budget_cycles < 0) return MXATTN_ERR_INVALID_ARG;
   if (o->causal != 0 && o->causal != 1) return MXATTN_ERR_INVALID_ARG;
+  if (o->format != MXATTN_FMT_MXFP4 && o->format != MXATTN_FMT_NVFP4) return MXATTN_ERR_INVALID_ARG;
+  if (o->causal && o->format == MXATTN_FMT_NVFP4) return MXATTN_ERR_UNSUPPORTED;  // NVFP4: full attention only
   return MXATTN_OK;
 }
 
@@ -70,20 +81,20 @@ struct Carve {
 };
 
 // Workspace carve-up: status block, then the packed Q operands (Nq tokens) and K/V operands (Nk).
-Carve carve(int B, int H, int Nq, int Nk, int d) {
+Carve carve(int B, int H, int Nq, int Nk, int d, int fmt) {
   Carve c;
   size_t off = kStatusBytes;
   c.q_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, Nq, d));
-  c.q_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, Nq, d));
+  c.q_scales = off; off = align256(off + qk_scale_bytes(B, H, Nq, d, fmt));
   c.k_codes = off; off = align256(off + mxattn_qk_codes_bytes(B, H, Nk, d));
-  c.k_scales = off; off = align256(off + mxattn_qk_scales_bytes(B, H, Nk, d));
+  c.k_scales = off; off = align256(off + qk_scale_bytes(B, H, Nk, d, fmt));
   c.v_codes = off; off = align256(off + mxattn_v_codes_bytes(B, H, Nk, d));
-  c.v_scales = off; off = align256(off + mxattn_v_scales_bytes(B, H, Nk, d));
+  c.v_scales = off; off = align256(off + v_scale_bytes(B, H, Nk, fmt));
   c.total = off;
   return c;
 }
 
-Carve carve(int B, int H, int N, int d) { return carve(B, H, N, N, d); }
+int fmt_of(const mxattn_opts* o) { return o != nullptr ? o->format : MXATTN_FMT_MXFP4; }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -112,6 +123,7 @@ void mxattn_opts_default(mxattn_opts* o) {
   o->workspace_bytes = 0;
   o->wait_budget_cycles = 0;
   o->causal = 0;
+  o->format = MXATTN_FMT_MXFP4;
 }
 
 size_t mxattn_qk_codes_bytes(int B, int H, int N, int d) {
@@ -134,7 +146,7 @@ size_t mxattn_v_scales_bytes(int B, int H, int N, int d) {
 size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts) {
   (void)opts;
   if (!sizes_ok(B, H, N, d)) return 0;
-  return carve(B, H, N, d).total;
+  return carve(B, H, N, N, d, fmt_of(opts)).total;
 }
 
 mxattn_status mxattn_workspace_init(const mxattn_opts* o, void* stream) {
@@ -161,6 +173,7 @@ mxattn_status mxattn_quantize_mxfp4(const void* x, int64_t rows, int64_t cols, i
   a.cols = cols;
   a.axis = group_axis;
   make_rule(o, &a.rule);
+  a.fmt = o->format;
   return launched(launch_quant_plain(a, o->dtype, as_stream(stream)));
 }
 
@@ -191,6 +204,7 @@ mxattn_status quant_qk(const void* q, const void* k, int B, int H, int Nq, int N
   a.rotate = o->rotate;
   a.hadamard_scale = (float)(1.0 / std::sqrt((double)d));
   make_rule(o, &a.rule);
+  a.fmt = o->format;
   return launched(launch_rotate_quant_qk(a, d, o->dtype, as_stream(stream)));
 }
 
@@ -218,6 +232,7 @@ mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mx
   a.BH = B * H;
   a.N = N;
   make_rule(o, &a.rule);
+  a.fmt = o->format;
   return launched(launch_quant_v(a, d, o->dtype, as_stream(stream)));
 }
 
@@ -255,6 +270,7 @@ mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const u
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
+  a.fmt = o->format;
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.causal = o->causal;
   a.dump = nullptr;
@@ -289,6 +305,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
+  if (o->format != MXATTN_FMT_MXFP4) return MXATTN_ERR_UNSUPPORTED;  // the dump reads MXFP4 tiles
   st = check_workspace(o, kStatusBytes);
   if (st != MXATTN_OK) return st;
   AttnArgs a{};
@@ -307,6 +324,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
   make_rule(o, &a.rule);
+  a.fmt = o->format;
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.causal = o->causal;
   a.dump = dump;
@@ -322,7 +340,7 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
-  const Carve c = carve(B, H, N, d);
+  const Carve c = carve(B, H, N, N, d, o->format);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
@@ -339,7 +357,7 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
 size_t mxattn_workspace_bytes_cross(int B, int H, int Nq, int Nk, int d, const mxattn_opts* opts) {
   (void)opts;
   if (!sizes_ok(B, H, Nq, d) || !sizes_ok(B, H, Nk, d)) return 0;
-  return carve(B, H, Nq, Nk, d).total;
+  return carve(B, H, Nq, Nk, d, fmt_of(opts)).total;
 }
 
 mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, int B, int H, int Nq, int Nk, int d,
@@ -350,7 +368,7 @@ mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, 
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
   if (o->causal) return MXATTN_ERR_UNSUPPORTED;  // no query/key position correspondence
-  const Carve c = carve(B, H, Nq, Nk, d);
+  const Carve c = carve(B, H, Nq, Nk, d, o->format);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
@@ -419,6 +437,7 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
+  if (o->format != MXATTN_FMT_MXFP4) return MXATTN_ERR_UNSUPPORTED;  // NVFP4: full attention only
   const VarlenCarve c = carve_varlen(nseq, H, tph, d);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
@@ -446,6 +465,7 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   qa.rotate = o->rotate;
   qa.hadamard_scale = (float)(1.0 / std::sqrt((double)d));
   qa.rule = rule;
+  qa.fmt = o->format;
   qa.vl = vl;
   st = launched(launch_rotate_quant_qk(qa, d, o->dtype, s));
   if (st != MXATTN_OK) return st;
@@ -457,6 +477,7 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   va.BH = H;
   va.N = T;
   va.rule = rule;
+  va.fmt = o->format;
   va.vl = vl;
   st = launched(launch_quant_v(va, d, o->dtype, s));
   if (st != MXATTN_OK) return st;
@@ -477,6 +498,7 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   a.tau = o->rescale_tau;
   a.pnq = o->pnq;
   a.rule = rule;
+  a.fmt = o->format;
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.dump = nullptr;
   a.dump_bh = a.dump_qt = -1;
@@ -502,7 +524,7 @@ struct HostPlan {
   size_t total;
 };
 
-HostPlan host_plan(int B, int H, int N, int d, int dtype) {
+HostPlan host_plan(int B, int H, int N, int d, int dtype, int fmt) {
   HostPlan p;
   p.BH = B * H;
   int nch = p.BH < kHostChunks ? p.BH : kHostChunks;
@@ -519,11 +541,11 @@ HostPlan host_plan(int B, int H, int N, int d, int dtype) {
     off = align256(off + (size_t)p.hc * p.head_bytes);
   }
   p.qc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
-  p.qs = off; off = align256(off + mxattn_qk_scales_bytes(1, p.hc, N, d));
+  p.qs = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
   p.kc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
-  p.ks = off; off = align256(off + mxattn_qk_scales_bytes(1, p.hc, N, d));
+  p.ks = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
   p.vc = off; off = align256(off + mxattn_v_codes_bytes(1, p.hc, N, d));
-  p.vs = off; off = align256(off + mxattn_v_scales_bytes(1, p.hc, N, d));
+  p.vs = off; off = align256(off + v_scale_bytes(1, p.hc, N, fmt));
   p.total = off;
   return p;
 }
@@ -534,7 +556,7 @@ extern "C" {
 
 size_t mxattn_workspace_bytes_host(int B, int H, int N, int d, const mxattn_opts* opts) {
   if (!sizes_ok(B, H, N, d)) return 0;
-  return host_plan(B, H, N, d, opts != nullptr ? opts->dtype : MXATTN_BF16).total;
+  return host_plan(B, H, N, d, opts != nullptr ? opts->dtype : MXATTN_BF16, fmt_of(opts)).total;
 }
 
 mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const void* v_host, int B, int H, int N,
@@ -544,7 +566,7 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
-  const HostPlan p = host_plan(B, H, N, d, o->dtype);
+  const HostPlan p = host_plan(B, H, N, d, o->dtype, o->format);
   st = check_workspace(o, p.total);
   if (st != MXATTN_OK) return st;
   uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);

@@ -42,7 +42,6 @@ constexpr int kBN = 64;         // keys per tile
 // of one CTA, and the masked variant (causal masking and/or a packed varlen batch).
 enum { kModeFull = 0, kModeDump = 1, kModeMasked = 2 };
 constexpr int kStages = 4;      // K/V shared-memory ring depth
-constexpr int kSfSlots = 3;     // K/V scale-factor slots in TMEM (reuse distance 3 tiles)
 // Warps 0-3 run the softmax (warp w reads TMEM lanes 32w..32w+31); the producer and the two MMA
 // issuers take three of the warps after them (where they sit was measured not to matter).
 #ifndef MXATTN_PRODUCER_WARP
@@ -74,8 +73,18 @@ constexpr long long kDrainBudgetCycles = 2000000000LL;
 // polynomial instead of MUFU.
 constexpr int kPolyWords = MXATTN_POLY_WORDS;
 
-template <int D>
+// NVF: the NVFP4 comparison format (E4M3 scales per 16 elements: one 512-byte scale atom per
+// 64 contraction elements, so Q/K carry D/64 atoms per tile and V one atom per 64-key tile).
+template <int D, bool NVF = false>
 struct Layout {
+  // K/V scale-factor slots in TMEM, reused every SLOTS tiles.  A slot's last reader, QK(j-SLOTS)
+  // or PV(j-SLOTS), is complete when it is overwritten for any SLOTS >= 2 (see the issuers);
+  // NVFP4's larger scale atoms fit the 256 columns with 2.
+  static constexpr int SLOTS = NVF ? 2 : 3;
+  static constexpr int QK_ATOMS = NVF ? D / 64 : 1;  // scale atoms of a Q tile / 128-key K tile
+  static constexpr int SFQ_BYTES = 512 * QK_ATOMS;
+  static constexpr int SFK_BYTES = 512 * QK_ATOMS;
+  static constexpr uint32_t ONES_SCALE = NVF ? 0x38383838u : 0x7F7F7F7Fu;  // 1.0 in E4M3 / E8M0
   // shared memory, byte offsets from a 1024-byte aligned base
   static constexpr int Q_BYTES = kBM * D / 2;
   static constexpr int K_BYTES = kBN * D / 2;
@@ -87,10 +96,10 @@ struct Layout {
   static constexpr int P_BYTES = kBM * kBN / 2;
   static constexpr int P_CODES = STAGE0 + kStages * STAGE_BYTES;  // two P buffers
   static constexpr int SF_Q = P_CODES + 2 * P_BYTES;
-  static constexpr int SF_P = SF_Q + 512;                         // two scale atoms
+  static constexpr int SF_P = SF_Q + SFQ_BYTES;                   // two scale atoms
   static constexpr int SF_ONES = SF_P + 2 * 512;  // scale atom of the ones rows (constant)
   static constexpr int SF_K = SF_ONES + 512;
-  static constexpr int SF_V = SF_K + kStages * 512;
+  static constexpr int SF_V = SF_K + kStages * SFK_BYTES;
   static constexpr int BARS = SF_V + kStages * 512;
   enum {
     B_Q = 0,
@@ -114,10 +123,11 @@ struct Layout {
   static constexpr uint32_t T_S = 0;
   static constexpr uint32_t T_O = 64;                      // O~: D columns, then l at column D
   static constexpr uint32_t T_SFQ = T_O + D + kOnesRows;
-  static constexpr uint32_t T_SFP = T_SFQ + 4;             // 2 x 4 columns
-  static constexpr uint32_t T_SFK = T_SFP + 8;             // kSfSlots x 4 columns
-  static constexpr uint32_t T_SFV = T_SFK + 4 * kSfSlots;  // kSfSlots x 8 columns (V atom + ones atom)
-  static_assert(T_SFV + 8 * kSfSlots <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t T_SFP = T_SFQ + 4 * QK_ATOMS;     // 2 x 4 columns
+  static constexpr uint32_t T_SFK = T_SFP + 8;                // SLOTS x (4 QK_ATOMS) columns
+  static constexpr uint32_t SFK_COLS = 4 * QK_ATOMS;
+  static constexpr uint32_t T_SFV = T_SFK + SFK_COLS * SLOTS;  // SLOTS x 8 columns (V atom + ones atom)
+  static_assert(T_SFV + 8 * SLOTS <= kTmemCols, "TMEM budget");
   static constexpr uint32_t QK_LAYOUT = D == 128 ? kLayoutSW64 : kLayoutSW32;
 };
 
@@ -185,9 +195,66 @@ __device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, i
   }
 }
 
-template <int D, int DT, bool PNQ, int MODE>
+// NVFP4 (comparison format) blocks of 16 keys: s[off..off+15] holds keys base..base+15.
+template <bool MASK>
+__device__ __forceinline__ float block16_max(const uint32_t (&s)[32], int off, int base, int valid) {
+  float m[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) {
+#pragma unroll
+    for (int k = 0; k < 2; k++) {
+      float v0 = __uint_as_float(s[off + i + 2 * k]), v1 = __uint_as_float(s[off + i + 2 * k + 1]);
+      if (MASK) {
+        v0 = base + i + 2 * k < valid ? v0 : -INFINITY;
+        v1 = base + i + 2 * k + 1 < valid ? v1 : -INFINITY;
+      }
+      m[k] = fmax3(m[k], v0, v1);
+    }
+  }
+  return fmaxf(m[0], m[1]);
+}
+
+// E2M1 codes of one block of 16: p = 2^(S*c - bias), 2 packed words (POLY: the second word's
+// exp2 from the FMA-pipe polynomial).
+template <bool MASK, bool SUM, bool POLY>
+__device__ __forceinline__ void block16_codes(const uint32_t (&s)[32], int off, int base, int valid, float c,
+                                              float bias, uint32_t* w, float& psum) {
+  const float2 cc = make_float2(c, c);
+  const float2 nb = make_float2(-bias, -bias);
+#pragma unroll
+  for (int q = 0; q < 2; q++) {
+    float p[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      const float2 x = __ffma2_rn(
+          make_float2(__uint_as_float(s[off + q * 8 + i]), __uint_as_float(s[off + q * 8 + i + 1])), cc, nb);
+      if (POLY && q == 1) {
+        const float2 y = exp2_poly2(x);
+        p[i] = y.x;
+        p[i + 1] = y.y;
+      } else {
+        p[i] = ex2_approx(x.x);
+        p[i + 1] = ex2_approx(x.y);
+      }
+      if (MASK) {
+        p[i] = base + q * 8 + i < valid ? p[i] : 0.f;
+        p[i + 1] = base + q * 8 + i + 1 < valid ? p[i + 1] : 0.f;
+      }
+      if (SUM) psum += p[i] + p[i + 1];
+    }
+    w[q] = cvt_e2m1x8(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7]);
+  }
+}
+
+// NVFP4 exponential tiles: P~ <= 1 is scaled by 448 * 6 before its blocks take their E4M3
+// scales, so that the block holding the running max (P~ = 1) gets scale 448 and code 6; the
+// factor cancels in O~ / l (both accumulate the scaled codes).
+constexpr float kLog2NvScale = 11.392317422778760f;  // log2(448 * 6)
+constexpr float kLog2E4m3Max = 8.807354922057604f;   // log2(448)
+
+template <int D, int DT, bool PNQ, int MODE, bool NVF>
 __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs a) {
-  using L = Layout<D>;
+  using L = Layout<D, NVF>;
   constexpr bool DUMP = MODE == kModeDump;
   constexpr bool MASKED = MODE == kModeMasked;
   constexpr int NV = PNQ ? D + kOnesRows : D;  // N of the PV MMA
@@ -260,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           off < (kBN / 2) / 4 ? 0x22222222u : 0u;
     }
     for (int i = threadIdx.x; i < 512 / 4; i += kThreads)
-      reinterpret_cast<uint32_t*>(smem + L::SF_ONES)[i] = i == 0 ? 0x7F7F7F7Fu : 0u;
+      reinterpret_cast<uint32_t*>(smem + L::SF_ONES)[i] = i == 0 ? L::ONES_SCALE : 0u;
     fence_proxy_async_smem();
   }
   if (warp == kQkWarp) {
@@ -278,9 +345,9 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     if (lane == 0) {
       bool ok = true;
       int issued = 0;
-      mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES + 512);
+      mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES + L::SFQ_BYTES);
       bulk_g2s(sb + L::Q_CODES, a.q_codes + q_tile * (size_t)L::Q_BYTES, L::Q_BYTES, bar(L::B_Q));
-      bulk_g2s(sb + L::SF_Q, a.q_scales + q_tile * 512, 512, bar(L::B_Q));
+      bulk_g2s(sb + L::SF_Q, a.q_scales + q_tile * L::SFQ_BYTES, L::SFQ_BYTES, bar(L::B_Q));
       for (int j = 0; j < TJ; j++) {
         const int s = j % kStages;
         if (j >= kStages) {
@@ -289,13 +356,14 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
         const uint32_t fb = bar(L::B_KV_FULL + s);
         const size_t t128 = k_tile0 + j / 2;
-        mbar_arrive_expect_tx(fb, L::K_BYTES + L::V_BYTES + 1024);
+        mbar_arrive_expect_tx(fb, L::K_BYTES + L::V_BYTES + L::SFK_BYTES + 512);
         bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES,
                  a.k_codes + (t128 * kBM + (j % 2) * kBN) * (size_t)(D / 2), L::K_BYTES, fb);
-        bulk_g2s(sb + L::SF_K + s * 512, a.k_scales + t128 * 512, 512, fb);
+        bulk_g2s(sb + L::SF_K + s * L::SFK_BYTES, a.k_scales + t128 * L::SFK_BYTES, L::SFK_BYTES, fb);
         bulk_g2s(sb + L::STAGE0 + s * L::STAGE_BYTES + L::K_BYTES,
                  a.v_codes + (v_tile0 + j) * (size_t)L::V_BYTES, L::V_BYTES, fb);
-        bulk_g2s(sb + L::SF_V + s * 512, a.v_scales + t128 * 512, 512, fb);
+        // V scales: MXFP4 one atom per 128-key tile (both 64-key halves), NVFP4 one per 64-key tile
+        bulk_g2s(sb + L::SF_V + s * 512, a.v_scales + (NVF ? v_tile0 + j : t128) * 512, 512, fb);
         issued = j + 1;
       }
       if (!ok) raise_abort(abort_flag, a.status, 1);
@@ -314,17 +382,20 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget));
     if (ok) {
       tc_fence_after();
-      if (leader) tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
+      if (leader)
+        for (int at = 0; at < L::QK_ATOMS; at++) tmem_cp_sf_atom(tmem + L::T_SFQ + 4 * at, sb + L::SF_Q + 512 * at);
       __syncwarp();
       const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
       for (int j = 0; j < TJ; j++) {
-        const int s = j % kStages, f = j % kSfSlots;
+        const int s = j % kStages, f = j % L::SLOTS;
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
         if (!ok) break;
         tc_fence_after();
-        // K scale slot f was last read by QK(j-3), complete since the softmax read S(j-3)
-        // before releasing it, which this warp waited for
-        if (leader) tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
+        // K scale slot f was last read by QK(j - SLOTS), complete since the softmax read that S
+        // before releasing it, which this warp waited for before issuing QK(j - 1)
+        if (leader)
+          for (int at = 0; at < L::QK_ATOMS; at++)
+            tmem_cp_sf_atom(tmem + L::T_SFK + L::SFK_COLS * f + 4 * at, sb + L::SF_K + L::SFK_BYTES * s + 512 * at);
         if (j > 0) {
           ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_S_FREE), (j - 1) & 1, abort_flag, a.wait_budget));
           if (!ok) break;
@@ -340,11 +411,17 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         if (leader) {
 #pragma unroll
           for (int kb = 0; kb < D / 64; kb++) {
-            // K block kb covers head dims 64kb..64kb+63: 32 bytes further along each row,
-            // scale bytes 2kb and 2kb+1 of each row's scale word.
-            mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
-                     mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
-                     tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
+            // K block kb covers head dims 64kb..64kb+63: 32 bytes further along each row;
+            // MXFP4: scale bytes 2kb and 2kb+1 of each row's scale word; NVFP4: scale atom kb.
+            // The K tile's 64 keys are rows 64(j&1).. of its 128-key atom: columns 2(j&1)..
+            if (NVF)
+              mma_nvf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2), nvf4_idesc(kBM, kBN),
+                       tmem + L::T_SFQ + 4 * kb, tmem + L::T_SFK + L::SFK_COLS * f + 4 * kb + 2 * (j & 1),
+                       kb > 0 ? 1u : 0u);
+            else
+              mma_mxf4(tmem + L::T_S, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
+                       mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
+                       tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
           }
           mma_commit(bar(L::B_S_FULL));
         }
@@ -360,11 +437,11 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
     // ------------------------------------------------------------------ PV issuer (same scheme)
     const bool leader = lane == 0;
     if (PNQ && leader)
-      for (int f = 0; f < kSfSlots; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
+      for (int f = 0; f < L::SLOTS; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
     __syncwarp();
     bool ok = true;
     for (int jp = 0; jp < TJ; jp++) {
-      const int sp = jp % kStages, fp = jp % kSfSlots, pb = jp & 1;
+      const int sp = jp % kStages, fp = jp % L::SLOTS, pb = jp & 1;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget));
       if (!ok) break;
       // V^(jp) landed with K^(jp), before S(jp) and so before P(jp); this warp also waits for the
@@ -376,18 +453,22 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       const uint64_t vdesc =
           smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
       if (leader) {
-        // P scale slot pb and V scale slot fp were last read by PV(jp-2) and PV(jp-3), complete
+        // P scale slot pb and V scale slot fp were last read by PV(jp-2) and PV(jp-SLOTS), complete
         // before S(jp) was committed, which the softmax saw before writing P(jp)
         tmem_cp_sf_atom(tmem + L::T_SFP + 4 * pb, sb + L::SF_P + 512 * pb);
         if (PNQ && D == 64) {
           // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
           // channels >= d are zero): give it scale 2^0 for all four key groups
-          *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * sp + 8) = 0x7F7F7F7Fu;
+          *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * sp + 8) = L::ONES_SCALE;
           fence_proxy_async_smem();
         }
         tmem_cp_sf_atom(tmem + L::T_SFV + 8 * fp, sb + L::SF_V + 512 * sp);
-        mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP + 4 * pb,
-                 tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
+        if (NVF)
+          mma_nvf4(tmem + L::T_O, pdesc, vdesc, nvf4_idesc(kBM, NV), tmem + L::T_SFP + 4 * pb, tmem + L::T_SFV + 8 * fp,
+                   jp > 0 ? 1u : 0u);
+        else
+          mma_mxf4(tmem + L::T_O, pdesc, vdesc, mxf4_idesc(kBM, NV, 0, 2 * (jp & 1)), tmem + L::T_SFP + 4 * pb,
+                   tmem + L::T_SFV + 8 * fp, jp > 0 ? 1u : 0u);
         mma_commit(bar(L::B_O_DONE + (jp & 1)));
         // QK(jp) read the stage too: complete, since the softmax saw S(jp) before P(jp)
         mma_commit(bar(L::B_KV_EMPTY + sp));
@@ -439,8 +520,14 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
 
       const int valid = FULL ? kBN : kmax - j * kBN;  // this row's keys in the tile (may be <= 0)
-      float gmax[2];
-      if (FULL) {
+      constexpr int NG = NVF ? 4 : 2;  // scale groups of the tile (MXFP4: 32 keys, NVFP4: 16)
+      float gmax[NG];
+      if constexpr (NVF) {
+        gmax[0] = block16_max<!FULL>(s0, 0, 0, valid);
+        gmax[1] = block16_max<!FULL>(s0, 16, 16, valid);
+        gmax[2] = block16_max<!FULL>(s1, 0, 32, valid);
+        gmax[3] = block16_max<!FULL>(s1, 16, 48, valid);
+      } else if (FULL) {
         gmax[0] = group_max<false>(s0, 0, valid);
         gmax[1] = group_max<false>(s1, 32, valid);
       } else {
@@ -451,7 +538,8 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       // maximum is taken as 2^((gmax - sm) * c): exactly 1 for the group that holds the running
       // max, as exp(0) is in the oracle, so scale rules whose boundaries sit on powers of two
       // (OCP, q = 4 or 8) decide it the same way.
-      const float mt_raw = fmaxf(gmax[0], gmax[1]);
+      float mt_raw = fmaxf(gmax[0], gmax[1]);
+      if constexpr (NVF) mt_raw = fmaxf(mt_raw, fmaxf(gmax[2], gmax[3]));
       const bool move = j == 0 || (mt_raw * c > m2 + a.tau);
       // O~ and l are rescaled by alpha = 2^(m_old - m_new) only when some row of the warp moves
       // its max (alpha = 1 elsewhere); tile 0 starts both at zero
@@ -462,13 +550,38 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       float alpha = 1.f;
       if (any_move && move) alpha = ex2_approx((sm_old - sm) * c);
 
-      uint32_t eb[2];  // E8M0 bytes
-      float bias[2];
+      uint32_t eb[NG];  // scale bytes (E8M0; NVFP4: E4M3)
+      float bias[NG];
+      float sc[NG];     // NVFP4: the scales' values
+      (void)sc;
+      if constexpr (NVF) {
+        // block b: y = P~ * 448 * 6, scale = E4M3(max y / 6) = E4M3(2^((gmax - sm) c + log2 448)),
+        // codes of y / scale = 2^(S c - m2 + log2(448 * 6) - log2 scale); a zero scale (a block
+        // far below the running max, or all masked) zeroes the block
 #pragma unroll
-      for (int g = 0; g < 2; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);
+        for (int g = 0; g < 4; g += 2) {
+          const uint32_t b2 = cvt_e4m3x2(ex2_approx((gmax[g] - sm) * c + kLog2E4m3Max),
+                                         ex2_approx((gmax[g + 1] - sm) * c + kLog2E4m3Max));
+          const float2 sv = e4m3x2_to_float2(b2);
+          eb[g] = b2 & 0xFFu;
+          eb[g + 1] = b2 >> 8;
+          sc[g] = sv.x;
+          sc[g + 1] = sv.y;
+          bias[g] = sv.x > 0.f ? m2 - kLog2NvScale + lg2_approx(sv.x) : INFINITY;
+          bias[g + 1] = sv.y > 0.f ? m2 - kLog2NvScale + lg2_approx(sv.y) : INFINITY;
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 2; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);
+      }
       uint32_t w[8];
-      float psum[2] = {0.f, 0.f};
-      if (FULL) {
+      float psum[NG] = {};
+      if constexpr (NVF) {
+        block16_codes<!FULL, !PNQ, false>(s0, 0, 0, valid, c, bias[0], w, psum[0]);
+        block16_codes<!FULL, !PNQ, true>(s0, 16, 16, valid, c, bias[1], w + 2, psum[1]);
+        block16_codes<!FULL, !PNQ, false>(s1, 0, 32, valid, c, bias[2], w + 4, psum[2]);
+        block16_codes<!FULL, !PNQ, true>(s1, 16, 48, valid, c, bias[3], w + 6, psum[3]);
+      } else if (FULL) {
         group_codes<false, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
         group_codes<false, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
       } else {
@@ -479,8 +592,13 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       s_ready = j + 1 < TJ && mbar_test(bar(L::B_S_FULL), (j + 1) & 1);
       if (!PNQ) {
         float lsum = 0.f;
+        if constexpr (NVF) {
 #pragma unroll
-        for (int g = 0; g < 2; g++) lsum += psum[g] * __uint_as_float(eb[g] << 23);  // byte 0: 2^-127 -> 0
+          for (int g = 0; g < 4; g++) lsum += psum[g] * sc[g];  // in units of y, as the PNQ sum
+        } else {
+#pragma unroll
+          for (int g = 0; g < 2; g++) lsum += psum[g] * __uint_as_float(eb[g] << 23);  // byte 0: 2^-127 -> 0
+        }
         l = alpha * l + lsum;
       }
 
@@ -516,8 +634,12 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       const int sw = (row >> 2) & 1;
       *reinterpret_cast<uint4*>(prow + (sw * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       *reinterpret_cast<uint4*>(prow + ((1 ^ sw) * 16)) = make_uint4(w[4], w[5], w[6], w[7]);
-      *reinterpret_cast<uint16_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
-          (uint16_t)(eb[0] | (eb[1] << 8));
+      if constexpr (NVF)
+        *reinterpret_cast<uint32_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
+            eb[0] | (eb[1] << 8) | (eb[2] << 16) | (eb[3] << 24);
+      else
+        *reinterpret_cast<uint16_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
+            (uint16_t)(eb[0] | (eb[1] << 8));
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -619,15 +741,17 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
   }
 }
 
-template <int D, int DT, bool PNQ>
+template <int D, int DT, bool PNQ, bool NVF>
 static cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
-  using L = Layout<D>;
+  using L = Layout<D, NVF>;
   // the diagnostic dump and the masking are separate instantiations, so the timed kernel carries
-  // none of them
+  // none of them; the NVFP4 comparison format runs full attention only
   const bool masked = a.causal || a.vl.cu_seqlens != nullptr;
-  auto kern = a.dump != nullptr ? mxattn_fwd_kernel<D, DT, PNQ, kModeDump>
-              : masked          ? mxattn_fwd_kernel<D, DT, PNQ, kModeMasked>
-                                : mxattn_fwd_kernel<D, DT, PNQ, kModeFull>;
+  if (NVF && (masked || a.dump != nullptr)) return cudaErrorNotSupported;
+  auto kern = NVF                 ? mxattn_fwd_kernel<D, DT, PNQ, kModeFull, NVF>
+              : a.dump != nullptr ? mxattn_fwd_kernel<D, DT, PNQ, kModeDump, false>
+              : masked            ? mxattn_fwd_kernel<D, DT, PNQ, kModeMasked, false>
+                                  : mxattn_fwd_kernel<D, DT, PNQ, kModeFull, false>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_SMEM);
   if (err != cudaSuccess) return err;
   const unsigned qtiles = a.vl.cu_seqlens != nullptr ? (unsigned)a.vl.tiles_per_head : (unsigned)((a.N + kBM - 1) / kBM);
@@ -636,13 +760,19 @@ static cudaError_t launch_attention_t(const AttnArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s) {
-  if (a.pnq) {
-    if (D == 128) return dtype == kBF16 ? launch_attention_t<128, kBF16, true>(a, s) : launch_attention_t<128, kFP32, true>(a, s);
-    return dtype == kBF16 ? launch_attention_t<64, kBF16, true>(a, s) : launch_attention_t<64, kFP32, true>(a, s);
-  }
-  if (D == 128) return dtype == kBF16 ? launch_attention_t<128, kBF16, false>(a, s) : launch_attention_t<128, kFP32, false>(a, s);
-  return dtype == kBF16 ? launch_attention_t<64, kBF16, false>(a, s) : launch_attention_t<64, kFP32, false>(a, s);
+template <int D, int DT>
+static cudaError_t launch_attention_d(const AttnArgs& a, cudaStream_t s) {
+  const bool nv = a.fmt == kFmtNVFP4;
+  if (a.pnq) return nv ? launch_attention_t<D, DT, true, true>(a, s) : launch_attention_t<D, DT, true, false>(a, s);
+  return nv ? launch_attention_t<D, DT, false, true>(a, s) : launch_attention_t<D, DT, false, false>(a, s);
 }
+
+cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s) {
+  if (D == 128) return dtype == kBF16 ? launch_attention_d<128, kBF16>(a, s) : launch_attention_d<128, kFP32>(a, s);
+  return dtype == kBF16 ? launch_attention_d<64, kBF16>(a, s) : launch_attention_d<64, kFP32>(a, s);
+}
+
+static_assert(Layout<128, true>::DYN_SMEM <= 113 * 1024 && Layout<128, false>::DYN_SMEM <= 113 * 1024,
+              "two CTAs per SM");
 
 }  // namespace mxattn

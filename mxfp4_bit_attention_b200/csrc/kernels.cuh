@@ -9,6 +9,9 @@
 namespace mxattn {
 
 enum { kBF16 = 0, kFP32 = 1 };
+// Element formats: the method's MXFP4 (32-element groups, E8M0 scale chosen by a ScaleRule) and
+// the NVFP4 comparison format (16-element blocks, E4M3 scale = E4M3(amax / 6)).
+enum { kFmtMXFP4 = 0, kFmtNVFP4 = 1 };
 
 // A packed batch of variable-length sequences ("varlen"): inputs and outputs are token-major
 // [T, H, d]; sequence s holds tokens cu_seqlens[s] .. cu_seqlens[s+1]-1 and is padded to whole
@@ -46,6 +49,7 @@ struct QKQuantArgs {
   float hadamard_scale;  // fl32(1/sqrt(d))
   ScaleRule rule;
   Varlen vl;
+  int fmt;
 };
 
 struct VQuantArgs {
@@ -55,6 +59,7 @@ struct VQuantArgs {
   int BH, N;             // varlen: BH = H, N = T
   ScaleRule rule;
   Varlen vl;
+  int fmt;
 };
 
 struct PlainQuantArgs {
@@ -64,6 +69,7 @@ struct PlainQuantArgs {
   int64_t rows, cols;
   int axis;
   ScaleRule rule;
+  int fmt;
 };
 
 // Per-block Qmax sweep (scale-rule diagnostic): boundaries q_k as ceiling rules.
@@ -99,6 +105,7 @@ struct AttnArgs {
   uint8_t* dump;         // optional diagnostic dump of one CTA (layout: see dump_layout below)
   int dump_bh, dump_qt;
   Varlen vl;             // varlen: BH = H, N = Nk = T
+  int fmt;               // kFmtNVFP4: the comparison format (full attention only)
 };
 
 // Diagnostic dump of the CTA (dump_bh, dump_qt), byte offsets for head dim D and T64 key tiles:

@@ -2,6 +2,8 @@
 // mbarriers, bulk async copies, tcgen05 (TMEM alloc, block-scaled MMA, commit,
 // smem->TMEM copy, TMEM loads/stores, fences) and the E2M1 conversions.
 #pragma once
+#include <cuda_fp16.h>
+
 #include <cstdint>
 
 namespace mxattn {
@@ -188,6 +190,24 @@ __host__ __device__ constexpr uint32_t mxf4_idesc(uint32_t M, uint32_t N, uint32
          ((M >> 4) << 24) | ((a_sf_id & 3u) << 29);
 }
 
+// The same for kind::mxf4nvf4 with 16-element blocks and UE4M3 scales (the NVFP4 comparison
+// format): scale format bit 23 = 0; a K = 64 instruction takes all four scale bytes of a
+// row's 32-bit TMEM word, so both scale-factor ids are 0.
+__host__ __device__ constexpr uint32_t nvf4_idesc(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T with per-32-element scales from TMEM.  One thread issues.
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
@@ -296,6 +316,22 @@ __device__ __forceinline__ uint32_t e2m1x32_sum_halves(uint32_t w0, uint32_t w1,
   return acc;
 }
 
+// E4M3 (FP8, bias 7, subnormals, largest finite 448) conversions for the NVFP4 block scales:
+// two fp32 -> two E4M3 bytes, round to nearest even, saturating (lo -> byte 0, hi -> byte 1).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(lo), "f"(hi));
+  return out;
+}
+
+// Two E4M3 bytes (byte 0 -> .x) -> their exact fp32 values (through f16, which holds every E4M3).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t bytes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)bytes));
+  return make_float2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))),
+                     __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
 // max of three fp32 values (one instruction on sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -330,6 +366,12 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 

@@ -40,6 +40,23 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid,
   }
 }
 
+// One NVFP4 block of 16 values (the comparison format): the scale is the E4M3 rounding of
+// fl32(amax / 6), each value is divided by it in fp32 (correctly rounded) and rounded to E2M1
+// with saturation; a scale that rounds to zero gives zero codes.  Returns the scale byte.
+__device__ __forceinline__ uint32_t nvfp4_block(const float* v, uint32_t* w) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t byte = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
+  const float s = e4m3x2_to_float2(byte).x;
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; i++) y[i] = s > 0.f ? __fdiv_rn(v[i], s) : 0.f;
+  w[0] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  w[1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  return byte;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Q/K: Hadamard rotation + quantization along d into the packed QK operand layout.
 // One thread per MX group (32 consecutive elements of a row, four 16-byte loads in flight), D/32
@@ -48,7 +65,7 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid,
 // Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K;
 // varlen: over H * tiles_per_head * 128 padded rows, each tile belonging to one sequence.
 // ------------------------------------------------------------------------------------------------
-template <int D, int DT>
+template <int D, int DT, bool NVF>
 __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
   constexpr int TPR = D / 32;                // threads per row = groups per row
   constexpr int ROWS = 256 / TPR;            // rows per block
@@ -133,24 +150,37 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
     }
   }
 
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-  const int e = shared_exponent(amax, a.rule);
-  const float inv = pow2_neg(e);
   uint32_t w[4];
+  int e = 0;
+  uint32_t nvb = 0;  // NVFP4: the two E4M3 scale bytes of the thread's blocks of 16
+  if (NVF) {
+    nvb = nvfp4_block(v, w) | (nvfp4_block(v + 16, w + 2) << 8);
+  } else {
+    float amax = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; q++)
-    w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
-                      __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
-                      __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
+    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+    e = shared_exponent(amax, a.rule);
+    const float inv = pow2_neg(e);
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+      w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
+                        __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
+                        __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
+  }
   if (!row_ok) return;
   const int s = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
   uint8_t* rowp = codes + (tile * 128 + r) * (D / 2);
   *reinterpret_cast<uint4*>(rowp + ((g ^ s) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
-  uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
-  atom[g] = (uint8_t)(e + 127);
-  if (D == 64) atom[g + 2] = 0;                           // unused scale slots
+  if (NVF) {
+    // D/64 scale atoms per tile, one per 64 dims (one K = 64 MMA): blocks 4a..4a+3 in the bytes
+    // of row r's word; this thread's blocks 2g, 2g+1 sit in atom g/2, bytes 2(g%2), 2(g%2)+1
+    uint8_t* atom = scales + tile * (512 * (D / 64)) + (g / 2) * 512 + (r % 32) * 16 + (r / 32) * 4;
+    *reinterpret_cast<uint16_t*>(atom + 2 * (g % 2)) = (uint16_t)nvb;
+  } else {
+    uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
+    atom[g] = (uint8_t)(e + 127);
+    if (D == 64) atom[g + 2] = 0;                         // unused scale slots
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -160,7 +190,7 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
 // Varlen: blocks over (head, 64-key tile of the packed tiles); each sequence's groups start at
 // its first token, and a sequence's tiles past its own keys are left unwritten.
 // ------------------------------------------------------------------------------------------------
-template <int D, int DT>
+template <int D, int DT, bool NVF>
 __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
   __shared__ float tile[64][D + 1];
   const bool vl = a.vl.cu_seqlens != nullptr;
@@ -208,6 +238,21 @@ __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
   __syncthreads();
   for (int item = t; item < 2 * D; item += 256) {
     const int c = item % D, h = item / D;
+    if (NVF) {
+      // two blocks of 16 keys; one scale atom per 64-key tile, keys 16b..16b+15 in byte b of
+      // channel c's word
+      float x[32];
+#pragma unroll
+      for (int i = 0; i < 32; i++) x[i] = tile[h * 32 + i][c];
+      uint32_t w[4];
+      const uint32_t b = nvfp4_block(x, w) | (nvfp4_block(x + 16, w + 2) << 8);
+      uint8_t* dst = a.v_codes + (vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      uint8_t* atom = a.v_scales + vtile * 512;
+      *reinterpret_cast<uint16_t*>(atom + (c % 32) * 16 + (c / 32) * 4 + 2 * h) = (uint16_t)b;
+      if (D == 64) *reinterpret_cast<uint16_t*>(atom + ((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 * h) = 0;
+      continue;
+    }
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(tile[h * 32 + i][c]));
@@ -239,11 +284,12 @@ __global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
 // Generic quantizer, plain layout: one thread per group of 32.
 // axis 0: groups along columns of a row; axis 1: groups along rows of a column (transposed out).
 // ------------------------------------------------------------------------------------------------
-template <int DT>
+template <int DT, bool NVF>
 __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
+  constexpr int G = NVF ? 16 : 32;  // elements per group / block
   const int64_t outer = a.axis == 0 ? a.rows : a.cols;
   const int64_t inner = a.axis == 0 ? a.cols : a.rows;
-  const int64_t ng = (inner + 31) / 32;
+  const int64_t ng = (inner + G - 1) / G;
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= outer * ng) return;
   // axis 1: consecutive threads take consecutive columns (coalesced); axis 0: consecutive groups
@@ -251,8 +297,8 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
   const int64_t g = a.axis == 0 ? gid % ng : gid / outer;
   float v[32];
 #pragma unroll
-  for (int i = 0; i < 32; i++) {
-    const int64_t in = g * 32 + i;
+  for (int i = 0; i < G; i++) {
+    const int64_t in = g * G + i;
     float x = 0.f;
     if (in < inner) {
       const int64_t idx = a.axis == 0 ? o * a.cols + in : in * a.cols + o;
@@ -262,6 +308,13 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
         x = reinterpret_cast<const float*>(a.x)[idx];
     }
     v[i] = x;
+  }
+  if (NVF) {
+    uint32_t w[2];
+    const uint32_t b = nvfp4_block(v, w);
+    *reinterpret_cast<uint2*>(a.codes + (o * ng + g) * 8) = make_uint2(w[0], w[1]);
+    a.scales[o * ng + g] = (uint8_t)b;
+    return;
   }
   float amax = 0.f;
 #pragma unroll
@@ -281,35 +334,54 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
 // ------------------------------------------------------------------------------------------------
 // Launchers
 // ------------------------------------------------------------------------------------------------
+template <int D, int DT>
+static void qk_launch(const QKQuantArgs& a, dim3 grid, cudaStream_t s) {
+  if (a.fmt == kFmtNVFP4) rotate_quant_qk_kernel<D, DT, true><<<grid, 256, 0, s>>>(a);
+  else rotate_quant_qk_kernel<D, DT, false><<<grid, 256, 0, s>>>(a);
+}
+
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
   const int64_t rows = a.vl.cu_seqlens != nullptr ? (int64_t)a.BH * a.vl.tiles_per_head * 128
                                                   : (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
   const int rows_per_block = 256 / (D / 32);
   dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
-  if (D == 128 && dtype == kBF16) rotate_quant_qk_kernel<128, kBF16><<<grid, 256, 0, s>>>(a);
-  else if (D == 128) rotate_quant_qk_kernel<128, kFP32><<<grid, 256, 0, s>>>(a);
-  else if (dtype == kBF16) rotate_quant_qk_kernel<64, kBF16><<<grid, 256, 0, s>>>(a);
-  else rotate_quant_qk_kernel<64, kFP32><<<grid, 256, 0, s>>>(a);
+  if (D == 128 && dtype == kBF16) qk_launch<128, kBF16>(a, grid, s);
+  else if (D == 128) qk_launch<128, kFP32>(a, grid, s);
+  else if (dtype == kBF16) qk_launch<64, kBF16>(a, grid, s);
+  else qk_launch<64, kFP32>(a, grid, s);
   return cudaGetLastError();
+}
+
+template <int D, int DT>
+static void v_launch(const VQuantArgs& a, unsigned blocks, cudaStream_t s) {
+  if (a.fmt == kFmtNVFP4) quant_v_kernel<D, DT, true><<<blocks, 256, 0, s>>>(a);
+  else quant_v_kernel<D, DT, false><<<blocks, 256, 0, s>>>(a);
 }
 
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s) {
   const unsigned blocks = (unsigned)((int64_t)a.BH * (a.vl.cu_seqlens != nullptr ? 2 * (int64_t)a.vl.tiles_per_head
                                                                                  : (a.N + 63) / 64));
-  if (D == 128 && dtype == kBF16) quant_v_kernel<128, kBF16><<<blocks, 256, 0, s>>>(a);
-  else if (D == 128) quant_v_kernel<128, kFP32><<<blocks, 256, 0, s>>>(a);
-  else if (dtype == kBF16) quant_v_kernel<64, kBF16><<<blocks, 256, 0, s>>>(a);
-  else quant_v_kernel<64, kFP32><<<blocks, 256, 0, s>>>(a);
+  if (D == 128 && dtype == kBF16) v_launch<128, kBF16>(a, blocks, s);
+  else if (D == 128) v_launch<128, kFP32>(a, blocks, s);
+  else if (dtype == kBF16) v_launch<64, kBF16>(a, blocks, s);
+  else v_launch<64, kFP32>(a, blocks, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant_plain(const PlainQuantArgs& a, int dtype, cudaStream_t s) {
   const int64_t outer = a.axis == 0 ? a.rows : a.cols;
   const int64_t inner = a.axis == 0 ? a.cols : a.rows;
-  const int64_t groups = outer * ((inner + 31) / 32);
+  const int G = a.fmt == kFmtNVFP4 ? 16 : 32;
+  const int64_t groups = outer * ((inner + G - 1) / G);
   const unsigned blocks = (unsigned)((groups + 255) / 256);
-  if (dtype == kBF16) quant_plain_kernel<kBF16><<<blocks, 256, 0, s>>>(a);
-  else quant_plain_kernel<kFP32><<<blocks, 256, 0, s>>>(a);
+  const bool nv = a.fmt == kFmtNVFP4;
+  if (dtype == kBF16) {
+    if (nv) quant_plain_kernel<kBF16, true><<<blocks, 256, 0, s>>>(a);
+    else quant_plain_kernel<kBF16, false><<<blocks, 256, 0, s>>>(a);
+  } else {
+    if (nv) quant_plain_kernel<kFP32, true><<<blocks, 256, 0, s>>>(a);
+    else quant_plain_kernel<kFP32, false><<<blocks, 256, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -36,7 +36,7 @@ def test_host_only_calls(lib):
     assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 64)
     assert abs(o.qmax - 7.25) < 1e-7 and abs(o.rescale_tau - 8.0) < 1e-7
     assert o.wait_budget_cycles == 0  # the library's default budget
-    assert o.causal == 0
+    assert o.causal == 0 and o.format == 0
     assert lib.mxattn_qk_codes_bytes(1, 2, 200, 128) == 2 * 2 * 128 * 64
     assert lib.mxattn_qk_scales_bytes(1, 2, 200, 128) == 2 * 2 * 512
     assert lib.mxattn_v_codes_bytes(1, 2, 200, 128) == 2 * 4 * 128 * 32
@@ -57,6 +57,13 @@ def test_host_only_calls(lib):
     assert lib.mxattn_workspace_bytes_varlen(3, 4, 1000, 128, ctypes.byref(o)) > one
     assert lib.mxattn_workspace_bytes_varlen(0, 4, 1000, 128, ctypes.byref(o)) == 0
     assert lib.mxattn_workspace_bytes_varlen(2, 4, 1000, 96, ctypes.byref(o)) == 0
+    # NVFP4: d/64 Q/K scale atoms per tile and one V atom per 64 keys
+    nv = binding.COpts()
+    lib.mxattn_opts_default(ctypes.byref(nv))
+    nv.format = 1
+    mx_b = lib.mxattn_workspace_bytes(1, 4, 1000, 128, ctypes.byref(o))
+    nv_b = lib.mxattn_workspace_bytes(1, 4, 1000, 128, ctypes.byref(nv))
+    assert nv_b - mx_b == 2 * 4 * 8 * 512 + 4 * (16 - 8) * 512
     assert lib.mxattn_status_string(5) == b"MXATTN_ERR_TIMEOUT"
 
 
@@ -89,6 +96,14 @@ def test_validation_rejects_before_enqueue(lib):
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 256, 64, 0.1, P, fake, None) == 2
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3  # no workspace
     o.causal = 0
+    o.format = 2
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
+    o.format = 1  # NVFP4 runs full attention only
+    o.causal = 1
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
+    o.causal = 0
+    assert lib.mxattn_forward_varlen(fake, fake, fake, fake, 2, 2, 100, 64, 0.1, P, fake, None) == 2
+    o.format = 0
     V = lib.mxattn_forward_varlen
     assert V(fake, fake, fake, fake, 0, 2, 100, 64, 0.1, P, fake, None) == 1     # nseq
     assert V(fake, fake, fake, fake, 2, 2, 100, 96, 0.1, P, fake, None) == 1     # d
