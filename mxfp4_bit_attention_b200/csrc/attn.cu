@@ -401,12 +401,6 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
           if (!ok) break;
           tc_fence_after();
         }
-        if (j >= 2) {
-          // S(j) also tells the softmax that P buffer j&1 (last read by PV(j-2)) is free: see
-          // PV(j-2) complete first.  Each O_DONE barrier is at most one phase away from it.
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget));
-          if (!ok) break;
-        }
         const uint64_t kdesc = smem_desc(sb + L::STAGE0 + s * L::STAGE_BYTES, 16, 8 * (D / 2), L::QK_LAYOUT);
         if (leader) {
 #pragma unroll
@@ -423,8 +417,16 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
                        mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ,
                        tmem + L::T_SFK + 4 * f + 2 * (j & 1), kb > 0 ? 1u : 0u);
           }
-          mma_commit(bar(L::B_S_FULL));
         }
+        if (j >= 2) {
+          // S(j) also tells the softmax that P buffer j&1 (last read by PV(j-2)) is free: see
+          // PV(j-2) complete before committing S(j) (the MMAs above, which touch neither P nor O~,
+          // already run meanwhile).  Each O_DONE barrier is at most one phase away from it.
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (leader) mma_commit(bar(L::B_S_FULL));
         __syncwarp();
       }
     }
@@ -440,29 +442,39 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       for (int f = 0; f < L::SLOTS; f++) tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f + 4, sb + L::SF_ONES);
     __syncwarp();
     bool ok = true;
+    // With three scale slots the V atom of tile jp is copied before P(jp) is awaited, off the path
+    // from P(jp) to PV(jp): its slot was last read by PV(jp-3), complete once S(jp-1) was committed
+    // (the QK issuer saw PV(jp-3) finish first), which P(jp-1) arriving implies.
+    constexpr bool kEarlyV = L::SLOTS >= 3;
+    auto copy_v_scales = [&](int sp, int fp) {
+      if (PNQ && D == 64) {
+        // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
+        // channels >= d are zero): give it scale 1 for all four key groups
+        *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * sp + 8) = L::ONES_SCALE;
+        fence_proxy_async_smem();
+      }
+      tmem_cp_sf_atom(tmem + L::T_SFV + 8 * fp, sb + L::SF_V + 512 * sp);
+    };
     for (int jp = 0; jp < TJ; jp++) {
       const int sp = jp % kStages, fp = jp % L::SLOTS, pb = jp & 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget));
-      if (!ok) break;
       // V^(jp) landed with K^(jp), before S(jp) and so before P(jp); this warp also waits for the
       // stage itself (it cannot have been refilled: that needs this warp's commit below)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + sp), (jp / kStages) & 1, abort_flag, a.wait_budget));
+      if (!ok) break;
+      tc_fence_after();
+      if (kEarlyV && leader) copy_v_scales(sp, fp);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (jp >> 1) & 1, abort_flag, a.wait_budget));
       if (!ok) break;
       tc_fence_after();
       const uint64_t pdesc = smem_desc(sb + L::P_CODES + pb * L::P_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
       const uint64_t vdesc =
           smem_desc(sb + L::STAGE0 + sp * L::STAGE_BYTES + L::K_BYTES, 16, 8 * (kBN / 2), kLayoutSW32);
       if (leader) {
-        // P scale slot pb and V scale slot fp were last read by PV(jp-2) and PV(jp-SLOTS), complete
-        // before S(jp) was committed, which the softmax saw before writing P(jp)
+        // P scale slot pb (and, without the early copy, V scale slot fp) were last read by PV(jp-2)
+        // (and PV(jp-SLOTS)), complete before S(jp) was committed, which the softmax saw before
+        // writing P(jp)
         tmem_cp_sf_atom(tmem + L::T_SFP + 4 * pb, sb + L::SF_P + 512 * pb);
-        if (PNQ && D == 64) {
-          // with d = 64 the ones row is B-operand row 64, inside the V scale atom (whose
-          // channels >= d are zero): give it scale 2^0 for all four key groups
-          *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * sp + 8) = L::ONES_SCALE;
-          fence_proxy_async_smem();
-        }
-        tmem_cp_sf_atom(tmem + L::T_SFV + 8 * fp, sb + L::SF_V + 512 * sp);
+        if (!kEarlyV) copy_v_scales(sp, fp);
         if (NVF)
           mma_nvf4(tmem + L::T_O, pdesc, vdesc, nvf4_idesc(kBM, NV), tmem + L::T_SFP + 4 * pb, tmem + L::T_SFV + 8 * fp,
                    jp > 0 ? 1u : 0u);
