@@ -132,3 +132,33 @@ def test_error_against_exact_attention_nvfp4_vs_mxfp4():
                                             "tau": tau, "pnq": pnq, "rel_l2": rel,
                                             "max_abs": float(err.abs().max())}))
     assert all(np.isfinite(list(table.values())))
+
+
+def test_nvfp4_cross_and_host_paths():
+    """The comparison format through cross-attention (keys of another length) against the oracle, and
+    through the host-buffer call against the device call, bit for bit."""
+    import torch
+    q, _, _ = _draw(2, 300, 128, "bf16", seed=41)
+    _, k, v = _draw(2, 1000, 128, "bf16", seed=42)
+    scale = float(np.float32(128 ** -0.5))
+    out = binding.mxattn_forward_cross(_dev(q, "bf16"), _dev(k, "bf16"), _dev(v, "bf16"), scale, NV)
+    torch.cuda.synchronize()
+    res = oracle.forward_rows(q, k, v, np.arange(300), scale, tau=8.0, fmt=oracle.FMT_NVFP4)
+    ref = oracle.round_to_bf16(res["out"])
+    got = out_to_numpy(out)[0]
+    tol = MAX_ABS_TOL + (2 / 3) * 1.1 * float(np.abs(v).max()) / res["l"][:, :, None]
+    assert rel_l2(got, ref) <= REL_L2_TOL and bool(np.all(np.abs(got - ref) <= tol))
+
+    qs, ks, vs = (_dev(x, "bf16") for x in _draw(6, 1000, 128, "bf16", seed=43))
+    dev = binding.mxattn_forward(qs, ks, vs, 0.088, NV)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (qs, ks, vs))
+    host = torch.empty_like(hq).pin_memory()
+    binding.mxattn_forward_host(hq, hk, hv, 0.088, NV, out=host)
+    torch.cuda.synchronize()
+    assert torch.equal(dev.cpu().view(torch.int16), host.view(torch.int16))
+
+
+def test_nvfp4_rejects_masking():
+    q, k, v = (_dev(x, "fp32") for x in _draw(1, 128, 64, "fp32", seed=2))
+    with pytest.raises(binding.MXAttnError):
+        binding.mxattn_forward(q, k, v, 0.125, binding.Opts(format=binding.FMT_NVFP4, causal=True))
