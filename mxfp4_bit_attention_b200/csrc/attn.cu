@@ -515,11 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       }
       tc_fence_after();
       uint32_t s0[32], s1[32];
-      tmem_ld32(tl + L::T_S, s0);
-      tmem_ld32(tl + L::T_S + 32, s1);
-      tmem_wait_ld();
-      pin32(s0);
-      pin32(s1);
+      tmem_ld64_wait(tl + L::T_S, tl + L::T_S + 32, s0, s1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_S_FREE));
