@@ -268,7 +268,8 @@ MXATTN_API mxattn_status mxattn_qmax_sweep(const void* x, int64_t rows, int64_t 
  * (the O~, l, m block starts at the next 16-byte boundary).  Used to measure
  * how many P^ codes differ from the oracle's and to study P~'s quantization
  * (per-block Qmax sweep, row-sum error decomposition); the paper has no
- * counterpart.
+ * counterpart.  Full attention in MXFP4 only: opts->causal or the NVFP4
+ * format return MXATTN_ERR_UNSUPPORTED.
  */
 MXATTN_API size_t mxattn_attention_dump_bytes(int N, int d);
 MXATTN_API mxattn_status mxattn_attention_mxfp4_dump(

@@ -306,6 +306,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
   if (o->format != MXATTN_FMT_MXFP4) return MXATTN_ERR_UNSUPPORTED;  // the dump reads MXFP4 tiles
+  if (o->causal) return MXATTN_ERR_UNSUPPORTED;                      // ... of full attention
   st = check_workspace(o, kStatusBytes);
   if (st != MXATTN_OK) return st;
   AttnArgs a{};

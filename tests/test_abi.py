@@ -92,6 +92,8 @@ def test_validation_rejects_before_enqueue(lib):
     o.causal = 2
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
     o.causal = 1  # causal masking needs a query/key position correspondence
+    assert lib.mxattn_attention_mxfp4_dump(fake, fake, fake, fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, 0, 0,
+                                           fake, None) == 2  # the dump runs full attention only
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 64, 0.1, P, fake, None) == 2
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 256, 64, 0.1, P, fake, None) == 2
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3  # no workspace
