@@ -366,7 +366,9 @@ def main():
     fp4_peak = bf16_peak * FP4_PER_BF16
     achieved = flops / (attn_ms_max * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp4_peak, "traffic": recorded_traffic(w.name),
+                "frac": achieved / fp4_peak,
+                # the recorded DRAM bytes are those of the full-attention MXFP4 kernel
+                "traffic": recorded_traffic(w.name) if (args.format == "mxfp4" and not args.causal) else None,
                 "kernel": "mxattn_fwd_kernel", "ms_per_launch": attn_ms_max,
                 "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
                 "frac_of_spec_9pf": achieved / 9000.0,
