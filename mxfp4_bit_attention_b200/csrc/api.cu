@@ -240,6 +240,35 @@ mxattn_status mxattn_quant_v(const void* v, int B, int H, int N, int d, const mx
 
 namespace {
 
+// Arguments of one attention launch on packed operands (no dump, no varlen table); the callers
+// set those fields themselves.
+AttnArgs attn_args(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes, const uint8_t* k_scales,
+                   const uint8_t* v_codes, const uint8_t* v_scales, int BH, int Nq, int Nk, float softmax_scale,
+                   const mxattn_opts* o, void* out, int* status) {
+  AttnArgs a{};
+  a.q_codes = q_codes;
+  a.q_scales = q_scales;
+  a.k_codes = k_codes;
+  a.k_scales = k_scales;
+  a.v_codes = v_codes;
+  a.v_scales = v_scales;
+  a.out = out;
+  a.status = status;
+  a.BH = BH;
+  a.N = Nq;
+  a.Nk = Nk;
+  a.causal = o->causal;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);  // softmax_scale * log2(e)
+  a.tau = o->rescale_tau;
+  a.pnq = o->pnq;
+  make_rule(o, &a.rule);
+  a.fmt = o->format;
+  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
+  a.dump = nullptr;
+  a.dump_bh = a.dump_qt = -1;
+  return a;
+}
+
 mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
                         const uint8_t* k_scales, const uint8_t* v_codes, const uint8_t* v_scales, int B, int H,
                         int Nq, int Nk, int d, float softmax_scale, const mxattn_opts* o, void* out, void* stream) {
@@ -254,27 +283,8 @@ mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const u
   const void* ptrs[] = {q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, out};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MXATTN_ERR_INVALID_ARG;
-  AttnArgs a{};
-  a.q_codes = q_codes;
-  a.q_scales = q_scales;
-  a.k_codes = k_codes;
-  a.k_scales = k_scales;
-  a.v_codes = v_codes;
-  a.v_scales = v_scales;
-  a.out = out;
-  a.status = reinterpret_cast<int*>(o->workspace);
-  a.BH = B * H;
-  a.N = Nq;
-  a.Nk = Nk;
-  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
-  a.tau = o->rescale_tau;
-  a.pnq = o->pnq;
-  make_rule(o, &a.rule);
-  a.fmt = o->format;
-  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
-  a.causal = o->causal;
-  a.dump = nullptr;
-  a.dump_bh = a.dump_qt = -1;
+  const AttnArgs a = attn_args(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, B * H, Nq, Nk, softmax_scale,
+                               o, out, reinterpret_cast<int*>(o->workspace));
   return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
 }
 
@@ -309,25 +319,8 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   if (o->causal) return MXATTN_ERR_UNSUPPORTED;                      // ... of full attention
   st = check_workspace(o, kStatusBytes);
   if (st != MXATTN_OK) return st;
-  AttnArgs a{};
-  a.q_codes = q_codes;
-  a.q_scales = q_scales;
-  a.k_codes = k_codes;
-  a.k_scales = k_scales;
-  a.v_codes = v_codes;
-  a.v_scales = v_scales;
-  a.out = out;
-  a.status = reinterpret_cast<int*>(o->workspace);
-  a.BH = B * H;
-  a.N = N;
-  a.Nk = N;
-  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
-  a.tau = o->rescale_tau;
-  a.pnq = o->pnq;
-  make_rule(o, &a.rule);
-  a.fmt = o->format;
-  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
-  a.causal = o->causal;
+  AttnArgs a = attn_args(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, B * H, N, N, softmax_scale, o, out,
+                         reinterpret_cast<int*>(o->workspace));
   a.dump = dump;
   a.dump_bh = dump_bh;
   a.dump_qt = dump_qt;
@@ -483,26 +476,8 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   st = launched(launch_quant_v(va, d, o->dtype, s));
   if (st != MXATTN_OK) return st;
 
-  AttnArgs a{};
-  a.q_codes = ws + c.q_codes;
-  a.q_scales = ws + c.q_scales;
-  a.k_codes = ws + c.k_codes;
-  a.k_scales = ws + c.k_scales;
-  a.v_codes = ws + c.v_codes;
-  a.v_scales = ws + c.v_scales;
-  a.out = out;
-  a.status = status;
-  a.BH = H;
-  a.N = a.Nk = T;
-  a.causal = o->causal;
-  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
-  a.tau = o->rescale_tau;
-  a.pnq = o->pnq;
-  a.rule = rule;
-  a.fmt = o->format;
-  a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
-  a.dump = nullptr;
-  a.dump_bh = a.dump_qt = -1;
+  AttnArgs a = attn_args(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes,
+                         ws + c.v_scales, H, T, T, softmax_scale, o, out, status);
   a.vl = vl;
   return launched(launch_attention(a, d, o->dtype, s));
 }
