@@ -289,16 +289,19 @@ MXATTN_API mxattn_status mxattn_forward(const void* q, const void* k, const void
  * The forward pass from and to HOST memory: q_host, k_host, v_host and
  * out_host are [B][H][N][d] of opts->dtype in host memory.  The B*H heads run
  * in up to 40 chunks (independent problems): chunk c's inputs are copied to
- * the device on an internal stream while chunk c-1 computes on `stream`, and
- * its output is copied back on another internal stream while chunk c+1
- * computes, so the transfers overlap the kernels.  Host buffers should be
- * page-locked (cudaHostAlloc / cudaHostRegister) for the copies to overlap;
- * pageable buffers give the same result without the overlap.  The workspace
- * (device, 256-byte aligned) holds mxattn_workspace_bytes_host(B, H, N, d,
- * opts) bytes (double-buffered staging of one chunk plus its packed
- * operands).  Every copy and kernel is ordered before the work enqueued on
- * `stream` afterwards: synchronize `stream` before reading out_host.  The
- * call creates two non-blocking streams and seven events and releases them
+ * the device on an internal stream while chunk c-1 computes, and its output
+ * is copied back on another internal stream while chunk c+1 computes, so the
+ * transfers overlap the kernels.  Even chunks compute on `stream`, odd ones
+ * on a third internal stream, each with its own packed-operand buffers, so
+ * that a chunk's kernels fill the SMs the previous chunk's last CTAs leave
+ * idle.  Host buffers should be page-locked (cudaHostAlloc /
+ * cudaHostRegister) for the copies to overlap; pageable buffers give the same
+ * result without the overlap.  The workspace (device, 256-byte aligned) holds
+ * mxattn_workspace_bytes_host(B, H, N, d, opts) bytes (double-buffered
+ * staging and packed operands of one chunk).  Every copy and kernel is
+ * ordered before the work enqueued on `stream` afterwards: synchronize
+ * `stream` before reading out_host.  The call creates three non-blocking
+ * streams and seven events and releases them
  * once their work completes; it allocates no memory.  Results equal
  * mxattn_forward's bit for bit.  Errors as for mxattn_forward (a failed CUDA
  * call returns MXATTN_ERR_CUDA).  The paper has no counterpart.

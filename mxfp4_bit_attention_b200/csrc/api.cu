@@ -496,7 +496,7 @@ struct HostPlan {
   int BH, hc, nch;               // heads, heads per chunk, chunks
   size_t head_bytes;             // one head of q, k, v or out
   size_t in_off[2], out_off[2];  // double-buffered q|k|v and out staging
-  size_t qc, qs, kc, ks, vc, vs; // packed operands of one chunk
+  size_t qc[2], qs[2], kc[2], ks[2], vc[2], vs[2];  // packed operands, one set per compute stream
   size_t total;
 };
 
@@ -516,12 +516,14 @@ HostPlan host_plan(int B, int H, int N, int d, int dtype, int fmt) {
     p.out_off[b] = off;
     off = align256(off + (size_t)p.hc * p.head_bytes);
   }
-  p.qc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
-  p.qs = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
-  p.kc = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
-  p.ks = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
-  p.vc = off; off = align256(off + mxattn_v_codes_bytes(1, p.hc, N, d));
-  p.vs = off; off = align256(off + v_scale_bytes(1, p.hc, N, fmt));
+  for (int b = 0; b < 2; b++) {
+    p.qc[b] = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
+    p.qs[b] = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
+    p.kc[b] = off; off = align256(off + mxattn_qk_codes_bytes(1, p.hc, N, d));
+    p.ks[b] = off; off = align256(off + qk_scale_bytes(1, p.hc, N, d, fmt));
+    p.vc[b] = off; off = align256(off + mxattn_v_codes_bytes(1, p.hc, N, d));
+    p.vs[b] = off; off = align256(off + v_scale_bytes(1, p.hc, N, fmt));
+  }
   p.total = off;
   return p;
 }
@@ -552,12 +554,15 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
   uint8_t* oh = reinterpret_cast<uint8_t*>(out_host);
   cudaStream_t s = as_stream(stream);
 
-  // copies in on s_in, compute on the caller's stream, copies out on s_out; every cross-stream
-  // order is an event, and the caller's stream finally waits for the last copies out
-  cudaStream_t s_in = nullptr, s_out = nullptr;
+  // Copies in on s_in, copies out on s_out, and the chunks' kernels alternately on the caller's
+  // stream and a second compute stream, each with its own operand buffers: a chunk's kernels start
+  // on the SMs that the previous chunk's last wave of CTAs leaves idle instead of after it.  Every
+  // cross-stream order is an event; the caller's stream finally waits for the last copies out.
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
   cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
   bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
             cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_c1, cudaStreamNonBlocking) == cudaSuccess &&
             cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess;
   for (int b = 0; ok && b < 2; b++)
     ok = cudaEventCreateWithFlags(&ev_in[b], cudaEventDisableTiming) == cudaSuccess &&
@@ -565,10 +570,13 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
          cudaEventCreateWithFlags(&ev_out[b], cudaEventDisableTiming) == cudaSuccess;
   // work already on the caller's stream comes first
   ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
-       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess && cudaStreamWaitEvent(s_c1, ev_start, 0) == cudaSuccess;
+  const cudaStream_t s_comp[2] = {s, s_c1};
   st = ok ? MXATTN_OK : MXATTN_ERR_CUDA;
   for (int c = 0; st == MXATTN_OK && c < p.nch; c++) {
     const int b = c & 1;
+    const cudaStream_t cs = s_comp[b];  // chunk c-2 ran on it too, with the same buffers
+    void* const csv = reinterpret_cast<void*>(cs);
     const int h0 = c * p.hc;
     const int hn = p.BH - h0 < p.hc ? p.BH - h0 : p.hc;
     const size_t bytes = (size_t)hn * p.head_bytes, src = (size_t)h0 * p.head_bytes;
@@ -582,19 +590,19 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
     if (cudaMemcpyAsync(qd, qh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
         cudaMemcpyAsync(kd, kh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
         cudaMemcpyAsync(vd, vh + src, bytes, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
-        cudaEventRecord(ev_in[b], s_in) != cudaSuccess || cudaStreamWaitEvent(s, ev_in[b], 0) != cudaSuccess) {
+        cudaEventRecord(ev_in[b], s_in) != cudaSuccess || cudaStreamWaitEvent(cs, ev_in[b], 0) != cudaSuccess) {
       st = MXATTN_ERR_CUDA;
       break;
     }
     // the output buffer b is free once chunk c-2's copy out has finished
-    if (c >= 2 && cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess) { st = MXATTN_ERR_CUDA; break; }
-    st = quant_qk(qd, kd, 1, hn, N, N, d, o, ws + p.qc, ws + p.qs, ws + p.kc, ws + p.ks, stream);
-    if (st == MXATTN_OK) st = mxattn_quant_v(vd, 1, hn, N, d, o, ws + p.vc, ws + p.vs, stream);
+    if (c >= 2 && cudaStreamWaitEvent(cs, ev_out[b], 0) != cudaSuccess) { st = MXATTN_ERR_CUDA; break; }
+    st = quant_qk(qd, kd, 1, hn, N, N, d, o, ws + p.qc[b], ws + p.qs[b], ws + p.kc[b], ws + p.ks[b], csv);
+    if (st == MXATTN_OK) st = mxattn_quant_v(vd, 1, hn, N, d, o, ws + p.vc[b], ws + p.vs[b], csv);
     if (st == MXATTN_OK)
-      st = attention(ws + p.qc, ws + p.qs, ws + p.kc, ws + p.ks, ws + p.vc, ws + p.vs, 1, hn, N, N, d, softmax_scale,
-                     o, od, stream);
+      st = attention(ws + p.qc[b], ws + p.qs[b], ws + p.kc[b], ws + p.ks[b], ws + p.vc[b], ws + p.vs[b], 1, hn, N, N,
+                     d, softmax_scale, o, od, csv);
     if (st != MXATTN_OK) break;
-    if (cudaEventRecord(ev_comp[b], s) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_comp[b], 0) != cudaSuccess ||
+    if (cudaEventRecord(ev_comp[b], cs) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_comp[b], 0) != cudaSuccess ||
         cudaMemcpyAsync(oh + src, od, bytes, cudaMemcpyDeviceToHost, s_out) != cudaSuccess ||
         cudaEventRecord(ev_out[b], s_out) != cudaSuccess) {
       st = MXATTN_ERR_CUDA;
@@ -615,6 +623,7 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
   if (ev_start) cudaEventDestroy(ev_start);
   if (s_in) cudaStreamDestroy(s_in);
   if (s_out) cudaStreamDestroy(s_out);
+  if (s_c1) cudaStreamDestroy(s_c1);
   return st;
 }
 
