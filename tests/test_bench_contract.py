@@ -1,0 +1,44 @@
+"""The bench's JSON contract, checked on the CPU through its reference arm (the oracle on a bounded
+sample) and its FLOP accounting."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench_module():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_attention_flops_full_and_causal():
+    from mxfp4_bit_attention_b200 import inputs
+    b = _bench_module()
+    w = inputs.WORKLOADS["720p"]
+    assert b.attention_flops(w, False) == 4.0 * 40 * 75600 * 75600 * 128
+    assert b.attention_flops(w, True) == 4.0 * 40 * (75600 * 75601 / 2) * 128
+    assert b.whole_job_tflops(2, 1e12, 1000.0) == pytest.approx(2.0)
+
+
+@pytest.mark.parametrize("extra", [[], ["--causal"]])
+def test_reference_arm_json_line(extra):
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--steps", "1", "--warmup", "1", "--cpu-sample-seconds", "0.5"] + extra
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["unit"] == "TFLOPS" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "tiny" and line["config"]["causal"] == bool(extra)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] > 0
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
