@@ -65,121 +65,185 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float* v, uint32_t* w) {
 // Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K;
 // varlen: over H * tiles_per_head * 128 padded rows, each tile belonging to one sequence.
 // ------------------------------------------------------------------------------------------------
+// Where padded row prow of the Q or K operand comes from: its row of the [rows, D] source (valid: a
+// real token; a padding row is quantized from zeros) and its packed tile and row within the tile.
+struct QKRow {
+  bool ok, valid;
+  int64_t src_row, tile;
+  int r;
+};
+
+__device__ __forceinline__ QKRow qk_row(const QKQuantArgs& a, int64_t prow, int64_t total, int64_t T128, int Nt) {
+  QKRow q;
+  q.ok = prow < total;
+  const int64_t bh = prow / (T128 * 128);
+  q.r = (int)(prow % 128);
+  q.tile = prow / 128;  // bh * T128 + tile within the head
+  if (a.vl.cu_seqlens != nullptr) {
+    // the tile's sequence and the row's token within it; tiles past the last sequence's are unused
+    const int gt = (int)(q.tile - bh * T128);
+    q.ok = q.ok && gt < __ldg(a.vl.tile_off + a.vl.nseq);
+    const int sq = q.ok ? varlen_sequence(a.vl, gt) : 0;
+    const int start = __ldg(a.vl.cu_seqlens + sq);
+    const int n = (gt - __ldg(a.vl.tile_off + sq)) * 128 + q.r;
+    q.valid = q.ok && n < __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    q.src_row = ((int64_t)start + n) * a.BH + bh;  // token-major [T, H, d]
+  } else {
+    const int tok = (int)(prow % (T128 * 128));
+    q.valid = q.ok && tok < Nt;
+    q.src_row = (int64_t)bh * Nt + tok;
+  }
+  return q;
+}
+
+// The 32 inputs of one thread's group as loaded (bf16: four 16-byte words; fp32: eight).
+template <int DT>
+struct GroupRaw {
+  uint4 w[DT == kBF16 ? 4 : 8];
+};
+
+template <int DT>
+__device__ __forceinline__ void load_group(const void* src, int64_t idx, bool valid, GroupRaw<DT>& raw) {
+  constexpr int NW = DT == kBF16 ? 4 : 8;
+  const uint4* p = DT == kBF16 ? reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + idx)
+                               : reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(src) + idx);
+#pragma unroll
+  for (int i = 0; i < NW; i++) raw.w[i] = valid ? p[i] : make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int DT>
+__device__ __forceinline__ void unpack_group(const GroupRaw<DT>& raw, float (&v)[32]) {
+  if (DT == kBF16) {
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const uint32_t w[4] = {raw.w[i].x, raw.w[i].y, raw.w[i].z, raw.w[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+        v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      v[4 * i] = __uint_as_float(raw.w[i].x);
+      v[4 * i + 1] = __uint_as_float(raw.w[i].y);
+      v[4 * i + 2] = __uint_as_float(raw.w[i].z);
+      v[4 * i + 3] = __uint_as_float(raw.w[i].w);
+    }
+  }
+}
+
+// Hadamard rotation of one row held by its TPR = D/32 lanes, 32 values each, in place: butterfly
+// stages h = 1..16 inside the thread, h = 32..D/2 across the row's lanes by shuffles, then the
+// multiply by fl32(1/sqrt(D)).  Every lane of the warp must take part (the shuffles are full-warp).
+template <int TPR>
+__device__ __forceinline__ void rotate_group(float (&v)[32], int g, float hadamard_scale) {
+  // Butterflies (x, y) -> (x + y, x - y), each result rounded once: x - y as fma(y, -1, x).
+  // From h = 2 on, neighbours i, i+1 pair up into f32x2 operations with the same roundings.
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float x = v[i], y = v[i + 1];
+    v[i] = __fadd_rn(x, y);
+    v[i + 1] = __fsub_rn(x, y);
+  }
+  const float2 minus1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      if ((i & h) == 0) {
+        const float2 x = make_float2(v[i], v[i + 1]), y = make_float2(v[i + h], v[i + h + 1]);
+        const float2 sum = __fadd2_rn(x, y), dif = __ffma2_rn(y, minus1, x);
+        v[i] = sum.x; v[i + 1] = sum.y;
+        v[i + h] = dif.x; v[i + h + 1] = dif.y;
+      }
+    }
+  }
+  // stages h = 32 .. D/2 across the TPR lanes of the row (lane bit = h / 32): the lower lane
+  // keeps x + y, the upper one y' = x - y, both as fma(own, +-1, other)
+#pragma unroll
+  for (int hb = 1; hb < TPR; hb <<= 1) {
+    const float sg = (g & hb) != 0 ? -1.f : 1.f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float o0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
+      const float o1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], hb);
+      const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), sg2, make_float2(o0, o1));
+      v[i] = r.x; v[i + 1] = r.y;
+    }
+  }
+  const float2 hs = make_float2(hadamard_scale, hadamard_scale);
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), hs);
+    v[i] = r.x; v[i + 1] = r.y;
+  }
+}
+
 template <int D, int DT, bool NVF>
 __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
   constexpr int TPR = D / 32;                // threads per row = groups per row
-  constexpr int ROWS = 256 / TPR;            // rows per block
+  constexpr int ROWS = 256 / TPR;            // rows per block and pass
   const int t = threadIdx.x;
   const int g = t % TPR;                     // group (and 16-byte code chunk) within the row
-  const int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;   // padded row id
   const int Nt = blockIdx.y == 0 ? a.N : a.Nk;  // tokens of this tensor
-  const bool vl = a.vl.cu_seqlens != nullptr;
-  const int64_t T128 = vl ? a.vl.tiles_per_head : (Nt + 127) / 128;  // 128-row tiles per head
+  const int64_t T128 = a.vl.cu_seqlens != nullptr ? a.vl.tiles_per_head : (Nt + 127) / 128;
   const int64_t total = (int64_t)a.BH * T128 * 128;
-  bool row_ok = prow < total;                // a row's threads are adjacent lanes of one warp
-  const int64_t bh = prow / (T128 * 128);
-  const int r = (int)(prow % 128);           // row within its tile
-  const int64_t tile = prow / 128;           // packed tile (bh * T128 + tile within the head)
-  bool valid;
-  int64_t src_row;                           // row of the [rows, D] source
-  if (vl) {
-    // the tile's sequence and the row's token within it; tiles past the last sequence's are unused
-    const int gt = (int)(tile - bh * T128);
-    row_ok = row_ok && gt < __ldg(a.vl.tile_off + a.vl.nseq);
-    const int sq = row_ok ? varlen_sequence(a.vl, gt) : 0;
-    const int start = __ldg(a.vl.cu_seqlens + sq);
-    const int n = (gt - __ldg(a.vl.tile_off + sq)) * 128 + r;
-    valid = row_ok && n < __ldg(a.vl.cu_seqlens + sq + 1) - start;
-    src_row = ((int64_t)start + n) * a.BH + bh;  // token-major [T, H, d]
-  } else {
-    const int tok = (int)(prow % (T128 * 128));
-    valid = row_ok && tok < Nt;
-    src_row = (int64_t)bh * Nt + tok;
-  }
-
   const void* src = blockIdx.y == 0 ? a.q : a.k;
   uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
   uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
 
-  float v[32];
-  const int64_t base = (valid ? src_row : 0) * D + g * 32;
-#pragma unroll
-  for (int c = 0; c < 4; c++) load8<DT>(src, base + c * 8, valid, *reinterpret_cast<float(*)[8]>(v + 8 * c));
-
-  if (a.rotate) {
-    // Butterflies (x, y) -> (x + y, x - y), each result rounded once: x - y as fma(y, -1, x).
-    // From h = 2 on, neighbours i, i+1 pair up into f32x2 operations with the same roundings.
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float x = v[i], y = v[i + 1];
-      v[i] = __fadd_rn(x, y);
-      v[i + 1] = __fsub_rn(x, y);
+  // Grid-stride over passes of ROWS rows (the pass count is the block's, so a row's lanes, which
+  // exchange values by shuffles, always run together); the next pass's inputs are loaded before
+  // this pass's rotation and quantization, so a load is in flight while the thread computes.
+  const int64_t stride = (int64_t)gridDim.x * ROWS;
+  int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;
+  QKRow row = qk_row(a, prow, total, T128, Nt);
+  GroupRaw<DT> raw;
+  load_group<DT>(src, (row.valid ? row.src_row : 0) * D + g * 32, row.valid, raw);
+  for (int64_t pass = (int64_t)blockIdx.x * ROWS; pass < total; pass += stride, prow += stride) {
+    const QKRow cur = row;
+    float v[32];
+    unpack_group<DT>(raw, v);
+    if (pass + stride < total) {
+      row = qk_row(a, prow + stride, total, T128, Nt);
+      load_group<DT>(src, (row.valid ? row.src_row : 0) * D + g * 32, row.valid, raw);
     }
-    const float2 minus1 = make_float2(-1.f, -1.f);
+    if (a.rotate) rotate_group<TPR>(v, g, a.hadamard_scale);
+    uint32_t w[4];
+    int e = 0;
+    uint32_t nvb = 0;  // NVFP4: the two E4M3 scale bytes of the thread's blocks of 16
+    if (NVF) {
+      nvb = nvfp4_block(v, w) | (nvfp4_block(v + 16, w + 2) << 8);
+    } else {
+      float amax = 0.f;
 #pragma unroll
-    for (int h = 2; h < 32; h <<= 1) {
+      for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+      e = shared_exponent(amax, a.rule);
+      const float inv = pow2_neg(e);
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        if ((i & h) == 0) {
-          const float2 x = make_float2(v[i], v[i + 1]), y = make_float2(v[i + h], v[i + h + 1]);
-          const float2 sum = __fadd2_rn(x, y), dif = __ffma2_rn(y, minus1, x);
-          v[i] = sum.x; v[i + 1] = sum.y;
-          v[i + h] = dif.x; v[i + h + 1] = dif.y;
-        }
-      }
+      for (int q = 0; q < 4; q++)
+        w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
+                          __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
+                          __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
     }
-    // stages h = 32 .. D/2 across the TPR lanes of the row (lane bit = h / 32): the lower lane
-    // keeps x + y, the upper one y' = x - y, both as fma(own, +-1, other)
-#pragma unroll
-    for (int hb = 1; hb < TPR; hb <<= 1) {
-      const float sg = (g & hb) != 0 ? -1.f : 1.f;
-      const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float o0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
-        const float o1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], hb);
-        const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), sg2, make_float2(o0, o1));
-        v[i] = r.x; v[i + 1] = r.y;
-      }
+    if (!cur.ok) continue;
+    const int r = cur.r;
+    const int sw = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
+    uint8_t* rowp = codes + (cur.tile * 128 + r) * (D / 2);
+    *reinterpret_cast<uint4*>(rowp + ((g ^ sw) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (NVF) {
+      // D/64 scale atoms per tile, one per 64 dims (one K = 64 MMA): blocks 4a..4a+3 in the bytes
+      // of row r's word; this thread's blocks 2g, 2g+1 sit in atom g/2, bytes 2(g%2), 2(g%2)+1
+      uint8_t* atom = scales + cur.tile * (512 * (D / 64)) + (g / 2) * 512 + (r % 32) * 16 + (r / 32) * 4;
+      *reinterpret_cast<uint16_t*>(atom + 2 * (g % 2)) = (uint16_t)nvb;
+    } else {
+      uint8_t* atom = scales + cur.tile * 512 + (r % 32) * 16 + (r / 32) * 4;
+      atom[g] = (uint8_t)(e + 127);
+      if (D == 64) atom[g + 2] = 0;                         // unused scale slots
     }
-    const float2 hs = make_float2(a.hadamard_scale, a.hadamard_scale);
-#pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), hs);
-      v[i] = r.x; v[i + 1] = r.y;
-    }
-  }
-
-  uint32_t w[4];
-  int e = 0;
-  uint32_t nvb = 0;  // NVFP4: the two E4M3 scale bytes of the thread's blocks of 16
-  if (NVF) {
-    nvb = nvfp4_block(v, w) | (nvfp4_block(v + 16, w + 2) << 8);
-  } else {
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-    e = shared_exponent(amax, a.rule);
-    const float inv = pow2_neg(e);
-#pragma unroll
-    for (int q = 0; q < 4; q++)
-      w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
-                        __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
-                        __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
-  }
-  if (!row_ok) return;
-  const int s = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
-  uint8_t* rowp = codes + (tile * 128 + r) * (D / 2);
-  *reinterpret_cast<uint4*>(rowp + ((g ^ s) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
-  if (NVF) {
-    // D/64 scale atoms per tile, one per 64 dims (one K = 64 MMA): blocks 4a..4a+3 in the bytes
-    // of row r's word; this thread's blocks 2g, 2g+1 sit in atom g/2, bytes 2(g%2), 2(g%2)+1
-    uint8_t* atom = scales + tile * (512 * (D / 64)) + (g / 2) * 512 + (r % 32) * 16 + (r / 32) * 4;
-    *reinterpret_cast<uint16_t*>(atom + 2 * (g % 2)) = (uint16_t)nvb;
-  } else {
-    uint8_t* atom = scales + tile * 512 + (r % 32) * 16 + (r / 32) * 4;
-    atom[g] = (uint8_t)(e + 127);
-    if (D == 64) atom[g + 2] = 0;                         // unused scale slots
   }
 }
 
@@ -344,7 +408,10 @@ cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaS
   const int64_t rows = a.vl.cu_seqlens != nullptr ? (int64_t)a.BH * a.vl.tiles_per_head * 128
                                                   : (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
   const int rows_per_block = 256 / (D / 32);
-  dim3 grid((unsigned)((rows + rows_per_block - 1) / rows_per_block), 2);
+  // enough blocks for every SM to hold several at once; each loops over the rest of the rows
+  const int64_t want = (rows + rows_per_block - 1) / rows_per_block;
+  constexpr int64_t kMaxBlocks = 148 * 8;
+  dim3 grid((unsigned)(want < kMaxBlocks ? want : kMaxBlocks), 2);
   if (D == 128 && dtype == kBF16) qk_launch<128, kBF16>(a, grid, s);
   else if (D == 128) qk_launch<128, kFP32>(a, grid, s);
   else if (dtype == kBF16) qk_launch<64, kBF16>(a, grid, s);
