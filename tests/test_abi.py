@@ -136,3 +136,44 @@ def test_package_import_does_not_need_the_library(monkeypatch):
     monkeypatch.setattr(binding, "lib_path", lambda: "/nonexistent/libmxattn.so")
     with pytest.raises(ImportError):
         binding.load()
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_workspace_sizes_follow_the_header(lib):
+    """The workspace sizes are the header's layouts added up: status block, then (varlen) the tile
+    table, then each packed operand, every piece 256-byte aligned."""
+    o = binding.COpts()
+    lib.mxattn_opts_default(ctypes.byref(o))
+    B, H, N, d = 2, 3, 1000, 128
+    t128, t64 = (N + 127) // 128, (N + 63) // 64
+    codes = B * H * t128 * 128 * d // 2
+    pieces = [codes, B * H * t128 * 512, codes, B * H * t128 * 512, B * H * t64 * d * 32, B * H * t128 * 512]
+    total = 256
+    for p in pieces:
+        total = _align256(total + p)
+    assert lib.mxattn_workspace_bytes(B, H, N, d, ctypes.byref(o)) == total
+    # NVFP4: d/64 Q/K scale atoms per tile, one V atom per 64 keys
+    o.format = 1
+    pieces = [codes, B * H * t128 * 512 * 2, codes, B * H * t128 * 512 * 2, B * H * t64 * d * 32, B * H * t64 * 512]
+    total = 256
+    for p in pieces:
+        total = _align256(total + p)
+    assert lib.mxattn_workspace_bytes(B, H, N, d, ctypes.byref(o)) == total
+    o.format = 0
+    # varlen: (T + 127 nseq) / 128 tiles per head, the tile table after the status block
+    nseq, T = 5, 1000
+    tph = (T + 127 * nseq) // 128
+    vcodes = H * tph * 128 * d // 2
+    pieces = [(nseq + 1) * 4, vcodes, H * tph * 512, vcodes, H * tph * 512, vcodes, H * tph * 512]
+    total = 256
+    for p in pieces:
+        total = _align256(total + p)
+    assert lib.mxattn_workspace_bytes_varlen(nseq, H, T, d, ctypes.byref(o)) == total
+    # the host-buffer call stages two chunks and keeps two sets of packed operands (two compute streams)
+    host = lib.mxattn_workspace_bytes_host(1, 40, 75600, 128, ctypes.byref(o))
+    head = 75600 * 128 * 2
+    one_set = lib.mxattn_workspace_bytes(1, 1, 75600, 128, ctypes.byref(o)) - 256
+    assert host >= 256 + 2 * 3 * head + 2 * head + 2 * one_set
