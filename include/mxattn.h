@@ -167,6 +167,12 @@ MXATTN_API size_t mxattn_qk_scales_bytes(int B, int H, int N, int d);
 MXATTN_API size_t mxattn_v_codes_bytes(int B, int H, int N, int d);
 MXATTN_API size_t mxattn_v_scales_bytes(int B, int H, int N, int d);
 
+/* The six sizes for the format in opts (MXFP4 or NVFP4), in the order q codes,
+ * q scales, k codes, k scales, v codes, v scales, written to sizes[0..5].
+ * Returns MXATTN_ERR_INVALID_ARG (sizes untouched) for invalid sizes or opts. */
+MXATTN_API mxattn_status mxattn_operand_bytes(int B, int H, int N, int d, const mxattn_opts* opts,
+                                              size_t* sizes);
+
 /* Zero the workspace status block (enqueued on stream). */
 MXATTN_API mxattn_status mxattn_workspace_init(const mxattn_opts* opts, void* stream);
 

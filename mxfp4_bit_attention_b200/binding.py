@@ -28,7 +28,7 @@ EXPORTS = (
     "mxattn_status_string", "mxattn_fp4_mma_probe", "mxattn_attention_dump_bytes",
     "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
     "mxattn_workspace_bytes_cross", "mxattn_forward_cross", "mxattn_workspace_bytes_host",
-    "mxattn_forward_host", "mxattn_workspace_bytes_varlen", "mxattn_forward_varlen",
+    "mxattn_forward_host", "mxattn_workspace_bytes_varlen", "mxattn_forward_varlen", "mxattn_operand_bytes",
 )
 
 
@@ -103,6 +103,7 @@ def load():
         "mxattn_forward_host": ([P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
         "mxattn_workspace_bytes_varlen": ([i32, i32, i32, i32, PO], sz),
         "mxattn_forward_varlen": ([P, P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
+        "mxattn_operand_bytes": ([i32, i32, i32, i32, PO, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -152,16 +153,11 @@ def _ptr(t):
 
 
 def operand_sizes(B: int, H: int, N: int, d: int, fmt: int = FMT_MXFP4) -> dict:
-    """Bytes of the packed operands; NVFP4 scales per the header (d/64 Q/K atoms per 128-row tile,
-    one V atom per 64-key tile)."""
-    L = load()
-    s = {"q_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "q_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
-         "k_codes": L.mxattn_qk_codes_bytes(B, H, N, d), "k_scales": L.mxattn_qk_scales_bytes(B, H, N, d),
-         "v_codes": L.mxattn_v_codes_bytes(B, H, N, d), "v_scales": L.mxattn_v_scales_bytes(B, H, N, d)}
-    if fmt == FMT_NVFP4:
-        s["q_scales"] = s["k_scales"] = s["q_scales"] * (d // 64)
-        s["v_scales"] = B * H * ((N + 63) // 64) * 512
-    return s
+    """Bytes of the packed operands for the element format (the library's mxattn_operand_bytes)."""
+    c = _copts(Opts(format=fmt), BF16)
+    sizes = (ctypes.c_size_t * 6)()
+    _check("mxattn_operand_bytes", load().mxattn_operand_bytes(B, H, N, d, ctypes.byref(c), sizes))
+    return dict(zip(("q_codes", "q_scales", "k_codes", "k_scales", "v_codes", "v_scales"), (int(x) for x in sizes)))
 
 
 def mxattn_workspace_bytes(B: int, H: int, N: int, d: int, opts: Opts | None = None) -> int:

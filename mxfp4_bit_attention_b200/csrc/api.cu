@@ -143,6 +143,16 @@ size_t mxattn_v_scales_bytes(int B, int H, int N, int d) {
   return (size_t)B * H * t128(N) * 512;
 }
 
+mxattn_status mxattn_operand_bytes(int B, int H, int N, int d, const mxattn_opts* opts, size_t* sizes) {
+  if (sizes == nullptr || !sizes_ok(B, H, N, d) || opts == nullptr) return MXATTN_ERR_INVALID_ARG;
+  if (opts->format != MXATTN_FMT_MXFP4 && opts->format != MXATTN_FMT_NVFP4) return MXATTN_ERR_INVALID_ARG;
+  sizes[0] = sizes[2] = mxattn_qk_codes_bytes(B, H, N, d);
+  sizes[1] = sizes[3] = qk_scale_bytes(B, H, N, d, opts->format);
+  sizes[4] = mxattn_v_codes_bytes(B, H, N, d);
+  sizes[5] = v_scale_bytes(B, H, N, opts->format);
+  return MXATTN_OK;
+}
+
 size_t mxattn_workspace_bytes(int B, int H, int N, int d, const mxattn_opts* opts) {
   (void)opts;
   if (!sizes_ok(B, H, N, d)) return 0;

@@ -172,6 +172,17 @@ def test_workspace_sizes_follow_the_header(lib):
     for p in pieces:
         total = _align256(total + p)
     assert lib.mxattn_workspace_bytes_varlen(nseq, H, T, d, ctypes.byref(o)) == total
+    # the per-operand sizes add up to the same layout
+    sizes = (ctypes.c_size_t * 6)()
+    o.format = 1
+    assert lib.mxattn_operand_bytes(B, H, N, d, ctypes.byref(o), sizes) == 0
+    assert list(sizes) == [codes, B * H * t128 * 1024, codes, B * H * t128 * 1024, B * H * t64 * d * 32,
+                           B * H * t64 * 512]
+    o.format = 3
+    assert lib.mxattn_operand_bytes(B, H, N, d, ctypes.byref(o), sizes) == 1
+    o.format = 0
+    assert lib.mxattn_operand_bytes(B, H, N, 96, ctypes.byref(o), sizes) == 1
+    assert lib.mxattn_operand_bytes(B, H, N, d, ctypes.byref(o), None) == 1
     # the host-buffer call stages two chunks and keeps two sets of packed operands (two compute streams)
     host = lib.mxattn_workspace_bytes_host(1, 40, 75600, 128, ctypes.byref(o))
     head = 75600 * 128 * 2
