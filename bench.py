@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4"],
                     help="element format: the method's MXFP4, or the NVFP4 comparison format")
+    ap.add_argument("--key-tile", type=int, default=64, choices=[64, 128],
+                    help="keys per online-softmax step (the attention kernel's key tile)")
     ap.add_argument("--causal", action="store_true",
                     help="causal self-attention; TFLOPS count the visible (query, key) pairs, N(N+1)/2 per head")
     return ap.parse_args()
@@ -286,7 +288,7 @@ def main():
     hq, hk, hv = (host_tensor(g[n]) for n in "qkv")
     del g
     q, k, v = (t.to(dev) for t in (hq, hk, hv))
-    opts = binding.Opts(causal=args.causal,
+    opts = binding.Opts(causal=args.causal, key_tile=args.key_tile,
                         format=binding.FMT_NVFP4 if args.format == "nvfp4" else binding.FMT_MXFP4)
     scale = float(np.float32(w.d ** -0.5))
     ws = binding.new_workspace(1, w.H, w.N, w.d, opts, dev)
@@ -385,7 +387,7 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "fp4(e2m1)+fp32 accumulate, bf16 in/out", "data": "synthetic",
                 "config": {"workload": w.name, "B": world, "H": w.H, "N": w.N, "d": w.d, "input_dtype": w.dtype,
-                           "key_tile": 64, "pnq": True, "rotate": True, "causal": args.causal,
+                           "key_tile": args.key_tile, "pnq": True, "rotate": True, "causal": args.causal,
                            "format": args.format,
                            "scale_rule": "UOS Qmax=7.25" if args.format == "mxfp4" else "E4M3(amax/6) per 16",
                            "rescale_tau": opts.rescale_tau, "parallelism": f"independent problems x{world}",

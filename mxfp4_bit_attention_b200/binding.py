@@ -226,18 +226,19 @@ def mxattn_attention_mxfp4(ops, B, H, N, d, softmax_scale, out, opts: Opts | Non
     return out
 
 
-def dump_layout(N: int, d: int) -> dict:
-    """Byte offsets of the diagnostic dump (mirrors the header's description)."""
-    T64 = (N + 63) // 64
-    p_codes = 2 * 128 * 64 * 4
-    p_scales = p_codes + T64 * 128 * 32
-    o = (p_scales + T64 * 128 * 2 + 15) // 16 * 16
+def dump_layout(N: int, d: int, key_tile: int = 64) -> dict:
+    """Byte offsets of the diagnostic dump for key tiles of key_tile keys (mirrors the header)."""
+    KT = key_tile
+    T = (N + KT - 1) // KT
+    p_codes = 2 * 128 * KT * 4
+    p_scales = p_codes + T * 128 * (KT // 2)
+    o = (p_scales + T * 128 * (KT // 32) + 15) // 16 * 16
     l = o + 128 * d * 4
     m = l + 128 * 4
     p_tilde = m + 128 * 4
-    m_tiles = p_tilde + T64 * 128 * 64 * 4
+    m_tiles = p_tilde + T * 128 * KT * 4
     return {"s": 0, "p_codes": p_codes, "p_scales": p_scales, "o": o, "l": l, "m": m, "p_tilde": p_tilde,
-            "m_tiles": m_tiles, "total": m_tiles + T64 * 128 * 4}
+            "m_tiles": m_tiles, "total": m_tiles + T * 128 * 4}
 
 
 def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, dump_qt=0, opts=None,
@@ -256,20 +257,21 @@ def mxattn_attention_mxfp4_dump(ops, B, H, N, d, softmax_scale, out, dump_bh=0, 
         _ptr(out), dump_bh, dump_qt, _ptr(dump), _stream(stream)))
     torch.cuda.synchronize()
     raw = dump.cpu().numpy()
-    L = dump_layout(N, d)
-    T64 = (N + 63) // 64
-    pc = raw[L["p_codes"]:L["p_scales"]].reshape(T64, 128, 32)
-    codes = np.empty((T64, 128, 64), np.uint8)
+    KT = int((opts or Opts()).key_tile)
+    L = dump_layout(N, d, KT)
+    T = (N + KT - 1) // KT
+    pc = raw[L["p_codes"]:L["p_scales"]].reshape(T, 128, KT // 2)
+    codes = np.empty((T, 128, KT), np.uint8)
     codes[..., 0::2] = pc & 0x0F
     codes[..., 1::2] = pc >> 4
-    return {"s": raw[:L["p_codes"]].view(np.float32).reshape(2, 128, 64),
+    return {"s": raw[:L["p_codes"]].view(np.float32).reshape(2, 128, KT),
             "p_codes": codes,
-            "p_scales": raw[L["p_scales"]:L["p_scales"] + T64 * 256].reshape(T64, 128, 2),
+            "p_scales": raw[L["p_scales"]:L["p_scales"] + T * 128 * (KT // 32)].reshape(T, 128, KT // 32),
             "o": raw[L["o"]:L["l"]].view(np.float32).reshape(128, d),
             "l": raw[L["l"]:L["m"]].view(np.float32).copy(),
             "m": raw[L["m"]:L["m"] + 512].view(np.float32).copy(),
-            "p_tilde": raw[L["p_tilde"]:L["m_tiles"]].view(np.float32).reshape(T64, 128, 64),
-            "m_tiles": raw[L["m_tiles"]:L["total"]].view(np.float32).reshape(T64, 128).copy()}
+            "p_tilde": raw[L["p_tilde"]:L["m_tiles"]].view(np.float32).reshape(T, 128, KT),
+            "m_tiles": raw[L["m_tiles"]:L["total"]].view(np.float32).reshape(T, 128).copy()}
 
 
 def mxattn_forward(q, k, v, softmax_scale=None, opts: Opts | None = None, out=None, workspace=None, stream=None):

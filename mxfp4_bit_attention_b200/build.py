@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 OUT = os.path.join(HERE, "libmxattn.so")
-SOURCES = ["api.cu", "quant.cu", "attn.cu", "probe.cu", "noalloc.cu", "sweep.cu", "varlen.cu"]
+SOURCES = ["api.cu", "quant.cu", "attn.cu", "attn_wide.cu", "probe.cu", "noalloc.cu", "sweep.cu", "varlen.cu"]
 HEADERS = ["ptx.cuh", "kernels.cuh"]
 
 

@@ -68,7 +68,8 @@ mxattn_status check_opts(const mxattn_opts* o) {
   if (o->pnq != 0 && o->pnq != 1) return MXATTN_ERR_INVALID_ARG;
   if (o->rotate != 0 && o->rotate != 1) return MXATTN_ERR_INVALID_ARG;
   if (!(o->rescale_tau >= 0.f && std::isfinite(o->rescale_tau))) return MXATTN_ERR_INVALID_ARG;
-  if (o->key_tile != 64) return o->key_tile == 128 ? MXATTN_ERR_UNSUPPORTED : MXATTN_ERR_INVALID_ARG;
+  if (o->key_tile != 64 && o->key_tile != 128) return MXATTN_ERR_INVALID_ARG;
+  if (o->key_tile == 128 && o->format == MXATTN_FMT_NVFP4) return MXATTN_ERR_UNSUPPORTED;
   if (o->wait_budget_cycles < 0) return MXATTN_ERR_INVALID_ARG;
   if (o->causal != 0 && o->causal != 1) return MXATTN_ERR_INVALID_ARG;
   if (o->format != MXATTN_FMT_MXFP4 && o->format != MXATTN_FMT_NVFP4) return MXATTN_ERR_INVALID_ARG;
@@ -276,7 +277,13 @@ AttnArgs attn_args(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_
   a.wait_budget = o->wait_budget_cycles > 0 ? o->wait_budget_cycles : kWaitBudgetCycles;
   a.dump = nullptr;
   a.dump_bh = a.dump_qt = -1;
+  a.key_tile = o->key_tile;
   return a;
+}
+
+// The attention kernel for the options' key tile width.
+cudaError_t launch_attn(const AttnArgs& a, int d, int dtype, cudaStream_t s) {
+  return a.key_tile == 128 ? launch_attention_wide(a, d, dtype, s) : launch_attention(a, d, dtype, s);
 }
 
 mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
@@ -295,7 +302,7 @@ mxattn_status attention(const uint8_t* q_codes, const uint8_t* q_scales, const u
     if (!aligned16(p)) return MXATTN_ERR_INVALID_ARG;
   const AttnArgs a = attn_args(q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, B * H, Nq, Nk, softmax_scale,
                                o, out, reinterpret_cast<int*>(o->workspace));
-  return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
+  return launched(launch_attn(a, d, o->dtype, as_stream(stream)));
 }
 
 }  // namespace
@@ -312,7 +319,9 @@ mxattn_status mxattn_attention_mxfp4(const uint8_t* q_codes, const uint8_t* q_sc
 
 size_t mxattn_attention_dump_bytes(int N, int d) {
   if (!sizes_ok(1, 1, N, d)) return 0;
-  return DumpLayout(d, (int)t64(N)).total;
+  // large enough for either key tile width
+  const size_t n64 = DumpLayout(d, (int)t64(N), 64).total, n128 = DumpLayout(d, (int)t128(N), 128).total;
+  return n64 > n128 ? n64 : n128;
 }
 
 mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t* q_scales, const uint8_t* k_codes,
@@ -334,7 +343,7 @@ mxattn_status mxattn_attention_mxfp4_dump(const uint8_t* q_codes, const uint8_t*
   a.dump = dump;
   a.dump_bh = dump_bh;
   a.dump_qt = dump_qt;
-  return launched(launch_attention(a, d, o->dtype, as_stream(stream)));
+  return launched(launch_attn(a, d, o->dtype, as_stream(stream)));
 }
 
 mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
@@ -344,10 +353,10 @@ mxattn_status mxattn_forward(const void* q, const void* k, const void* v, int B,
   if (!(softmax_scale > 0.f && std::isfinite(softmax_scale))) return MXATTN_ERR_INVALID_ARG;
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
   const Carve c = carve(B, H, N, N, d, o->format);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
   uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
   st = mxattn_hadamard_quant_qk(q, k, B, H, N, d, o, ws + c.q_codes, ws + c.q_scales, ws + c.k_codes,
                                 ws + c.k_scales, stream);
@@ -372,10 +381,10 @@ mxattn_status mxattn_forward_cross(const void* q, const void* k, const void* v, 
   mxattn_status st = check_opts(o);
   if (st != MXATTN_OK) return st;
   if (o->causal) return MXATTN_ERR_UNSUPPORTED;  // no query/key position correspondence
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
   const Carve c = carve(B, H, Nq, Nk, d, o->format);
   st = check_workspace(o, c.total);
   if (st != MXATTN_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return MXATTN_ERR_INVALID_ARG;
   uint8_t* ws = reinterpret_cast<uint8_t*>(o->workspace);
   st = quant_qk(q, k, B, H, Nq, Nk, d, o, ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, stream);
   if (st != MXATTN_OK) return st;
@@ -489,7 +498,7 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
   AttnArgs a = attn_args(ws + c.q_codes, ws + c.q_scales, ws + c.k_codes, ws + c.k_scales, ws + c.v_codes,
                          ws + c.v_scales, H, T, T, softmax_scale, o, out, status);
   a.vl = vl;
-  return launched(launch_attention(a, d, o->dtype, s));
+  return launched(launch_attn(a, d, o->dtype, s));
 }
 
 }  // extern "C"

@@ -106,29 +106,31 @@ struct AttnArgs {
   int dump_bh, dump_qt;
   Varlen vl;             // varlen: BH = H, N = Nk = T
   int fmt;               // kFmtNVFP4: the comparison format (full attention only)
+  int key_tile;          // 64 or 128 keys per online-softmax step
 };
 
-// Diagnostic dump of the CTA (dump_bh, dump_qt), byte offsets for head dim D and T64 key tiles:
-//   [0, 64K)               S of key tiles 0 and 1, fp32 [2][128][64] (as read from TMEM)
-//   P codes                [T64][128][32] bytes, logical key order (element 2i in the low nibble)
-//   P scales               [T64][128][2] bytes (E8M0 of key groups 0 and 1 of the tile)
+// Diagnostic dump of the CTA (dump_bh, dump_qt), byte offsets for head dim D, key tiles of KT keys
+// (64 or 128) and T = ceil(N / KT) tiles:
+//   [0, 8 KT * 128)        S of key tiles 0 and 1, fp32 [2][128][KT] (as read from TMEM)
+//   P codes                [T][128][KT/2] bytes, logical key order (element 2i in the low nibble)
+//   P scales               [T][128][KT/32] bytes (E8M0 of the tile's 32-key groups)
 //   O accumulator          [128][D] fp32, before the division by l
 //   l, m                   [128] fp32 each (m in log2 units: running max of S * scale * log2 e)
-//   P~                     [T64][128][64] fp32: 2^(S * scale * log2 e - m) with the running max m
+//   P~                     [T][128][KT] fp32: 2^(S * scale * log2 e - m) with the running max m
 //                          of that tile (0 for keys past N), the unquantized exponential tile
-//   m of every tile        [T64][128] fp32, the running max (log2 units) after each tile's update
+//   m of every tile        [T][128] fp32, the running max (log2 units) after each tile's update
 struct DumpLayout {
   size_t s, p_codes, p_scales, o, l, m, p_tilde, m_tiles, total;
-  __host__ __device__ DumpLayout(int D, int T64) {
+  __host__ __device__ DumpLayout(int D, int T, int KT = 64) {
     s = 0;
-    p_codes = 2 * 128 * 64 * 4;
-    p_scales = p_codes + (size_t)T64 * 128 * 32;
-    o = (p_scales + (size_t)T64 * 128 * 2 + 15) / 16 * 16;
+    p_codes = (size_t)2 * 128 * KT * 4;
+    p_scales = p_codes + (size_t)T * 128 * (KT / 2);
+    o = (p_scales + (size_t)T * 128 * (KT / 32) + 15) / 16 * 16;
     l = o + (size_t)128 * D * 4;
     m = l + 128 * 4;
     p_tilde = m + 128 * 4;
-    m_tiles = p_tilde + (size_t)T64 * 128 * 64 * 4;
-    total = m_tiles + (size_t)T64 * 128 * 4;
+    m_tiles = p_tilde + (size_t)T * 128 * KT * 4;
+    total = m_tiles + (size_t)T * 128 * 4;
   }
 };
 
@@ -141,6 +143,7 @@ cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s
 cudaError_t launch_quant_plain(const PlainQuantArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_qmax_sweep(const SweepArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s);
+cudaError_t launch_attention_wide(const AttnArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_fp4_mma_probe(int ctas, int iters, int n, int* status, cudaStream_t s);
 cudaError_t launch_varlen_tiles(const int* cu_seqlens, int nseq, int T, int* tile_off, int* status, cudaStream_t s);
 

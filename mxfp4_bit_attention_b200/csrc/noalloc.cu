@@ -49,6 +49,16 @@ extern "C" MXATTN_API mxattn_status mxattn_forward_noalloc(const void* q, const 
   const size_t need = mxattn_workspace_bytes(B, H, N, d, opts);
   if (need == 0) return MXATTN_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return MXATTN_ERR_WORKSPACE;  // problem larger than the fixed scratch
+  // Every argument check of mxattn_forward runs before anything is enqueued: mxattn_forward's own
+  // checks would come after the status-block reset below.  A dry run with a non-null stand-in for
+  // the workspace and a zero size checks everything but the workspace, which is ours.
+  {
+    mxattn_opts probe = *opts;
+    probe.workspace = nullptr;
+    probe.workspace_bytes = 0;
+    const mxattn_status st = mxattn_forward(q, k, v, B, H, N, d, softmax_scale, &probe, out, stream);
+    if (st != MXATTN_ERR_WORKSPACE) return st;  // an argument error (a missing workspace is all it may lack)
+  }
   void* scratch = nullptr;
   const mxattn_status st = scratch_for_current_device(&scratch);
   if (st != MXATTN_OK) return st;

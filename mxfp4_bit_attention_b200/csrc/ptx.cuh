@@ -300,6 +300,39 @@ __device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr0, uint32_t taddr1,
       : "memory");
 }
 
+// 128 consecutive 32-bit columns in one load, waited for in the same statement (the outputs exist
+// only after the wait, so no use can be scheduled above it).
+__device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
+      "%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,"
+      "%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,"
+      "%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,"
+      "%126,%127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+        "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]),
+        "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]),
+        "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]),
+        "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void pin32(uint32_t (&r)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; i++) pin1(r[i]);
@@ -393,6 +426,54 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// fma with the result clamped to [0, 1] (one instruction)
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// bits(q) + bits(t) * 2^23 in one integer multiply-add: adds the integer held in the low bits of
+// t to q's exponent field.
+__device__ __forceinline__ float add_exponent(float q, float t) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r) : "r"(__float_as_uint(t)), "r"(__float_as_uint(q)));
+  return __uint_as_float(r);
+}
+
+// A stand-in for 2^u that gives the same E2M1 code as 2^u under cvt.rn.satfinite.e2m1x2 (round to
+// nearest even, saturating at 6), for a pair of arguments given as w = clamp((u + 4) / 8, 0, 1),
+// computed on the FMA pipe alone.
+//
+// The E2M1 code of a positive value depends only on where it lies against the grid midpoints
+// 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5.  Writing u = k + f (k = floor u, f in [0, 1)), every
+// midpoint is 2^k times one of 1 (k = -2: the 0.25 tie, which rounds to 0), 1.25, 1.5 (k = -1:
+// 0.75) or 1.75.  So the value 2^k * q(f) gets the code of 2^u whenever q is increasing on [0, 1),
+// meets 2^f at f = log2 1.25, log2 1.5 and log2 1.75, stays above 1 at f = 0 and below 2 as f -> 1
+// (then the step at each integer k crosses 0.25 only at u = -2 exactly and crosses no other
+// midpoint).  The quadratic through those three points does all of this: q(0) = 1.0114,
+// q(1) = 1.9952, q' > 0.  Arguments below -4 map to k = -4 (2^-4 * q < 0.25: code 0); the
+// clamp also keeps k in a range where adding it to the exponent field cannot wrap.  The result
+// is a code-exact stand-in, not an accurate exponential: use it only in front of the E2M1
+// conversion.
+constexpr float kQuadC0 = 1.0114069778f;
+constexpr float kQuadC1 = 0.6259469002f;
+constexpr float kQuadC2 = 0.3578150505f;
+constexpr float kFloorMagic = 12582912.f;  // 1.5 * 2^23: integers in the low mantissa bits
+
+__device__ __forceinline__ float2 e2m1_exp2_stand_in(float2 w) {
+  const float2 m4 = make_float2(kFloorMagic - 4.f, kFloorMagic - 4.f);
+  const float2 eight = make_float2(8.f, 8.f);
+  // t = M + floor(8w - 4): the sum is positive, so rounding toward zero is rounding down
+  const float2 t = __ffma2_rz(w, eight, m4);
+  const float2 nk = __ffma2_rn(t, make_float2(-1.f, -1.f), m4);  // -floor(8w), exact
+  const float2 f = __ffma2_rn(w, eight, nk);                       // 8w - floor(8w), exact
+  float2 q = __ffma2_rn(f, make_float2(kQuadC2, kQuadC2), make_float2(kQuadC1, kQuadC1));
+  q = __ffma2_rn(q, f, make_float2(kQuadC0, kQuadC0));
+  // the low bits of t hold k (the constant's own bits shift out of the 32-bit product)
+  return make_float2(add_exponent(q.x, t.x), add_exponent(q.y, t.y));
 }
 
 __device__ __forceinline__ float lg2_approx(float x) {

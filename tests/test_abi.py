@@ -83,9 +83,13 @@ def test_validation_rejects_before_enqueue(lib):
     assert lib.mxattn_forward_cross(fake, fake, fake, 1, 1, 256, 100, 64, 0.1, P, fake, None) == 3  # no workspace
     assert lib.mxattn_forward_host(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3       # no workspace
     assert lib.mxattn_forward_host(None, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1       # null
-    o.key_tile = 128
+    o.key_tile = 128  # supported: only the workspace is missing
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 3
+    o.key_tile = 96
+    assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
+    o.key_tile, o.format = 128, 1  # NVFP4 runs with 64-key tiles only
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 2
-    o.key_tile = 64
+    o.key_tile, o.format = 64, 0
     o.wait_budget_cycles = -5
     assert lib.mxattn_forward(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1
     o.wait_budget_cycles = 0
@@ -188,3 +192,19 @@ def test_workspace_sizes_follow_the_header(lib):
     head = 75600 * 128 * 2
     one_set = lib.mxattn_workspace_bytes(1, 1, 75600, 128, ctypes.byref(o)) - 256
     assert host >= 256 + 2 * 3 * head + 2 * head + 2 * one_set
+
+
+def test_noalloc_checks_arguments_before_enqueueing():
+    """mxattn_forward_noalloc runs every argument check of mxattn_forward before it touches the
+    device: on this CPU-only host any device call would fail with MXATTN_ERR_CUDA, so an argument
+    error must come back as MXATTN_ERR_INVALID_ARG."""
+    lib = binding.load()
+    o = binding.COpts()
+    lib.mxattn_opts_default(ctypes.byref(o))
+    P = ctypes.byref(o)
+    fake, odd = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
+    assert lib.mxattn_forward_noalloc(odd, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1      # misaligned q
+    assert lib.mxattn_forward_noalloc(fake, fake, fake, 1, 1, 256, 64, -1.0, P, fake, None) == 1    # scale
+    assert lib.mxattn_forward_noalloc(fake, fake, None, 1, 1, 256, 64, 0.1, P, fake, None) == 1     # null v
+    o.pnq = 3
+    assert lib.mxattn_forward_noalloc(fake, fake, fake, 1, 1, 256, 64, 0.1, P, fake, None) == 1     # options

@@ -199,3 +199,30 @@ def test_varlen_sequences_are_independent():
     one = oracle.forward_rows(q.transpose(1, 0, 2).copy(), k.transpose(1, 0, 2).copy(),
                               v.transpose(1, 0, 2).copy(), rows, 0.09, tau=8.0)["out"].transpose(1, 0, 2)
     np.testing.assert_array_equal(whole, one)
+
+
+@pytest.mark.parametrize("key_tile", [64, 128])
+@pytest.mark.parametrize("tau", [8.0, 3.0])
+def test_lazy_max_moves_only_past_tau_log2_units(key_tile, tau):
+    """The lazy running max (Pith review page, axioms ledger: the FlashAttention-2 running max;
+    Fig. 4B) moves only when a tile's max exceeds it by more than tau in log2 units.  Two tiles:
+    tile 0 has scores 0, tile 1 one key whose score sits eps below or above tau * ln 2 (natural
+    units).  With eps far below the distance between the log2 and natural readings of tau (a
+    factor ln 2), a units mistake moves the max in both cases or in neither."""
+    d, T = 64, key_tile
+    q = np.zeros((1, d))
+    q[0, 0] = 1.0
+    k = np.zeros((2 * T, d))
+    v = np.random.default_rng(0).standard_normal((2 * T, d))
+    eps = 1e-4
+    for sign, moves in ((-1, False), (+1, True)):
+        b = float(np.float32(tau * math.log(2) * (1 + sign * eps)))
+        k[T, 0] = b
+        r = oracle.attention_rows(q, k, v, 1.0, key_tile, tau=tau, codes=True)
+        assert r["m"][0] == (b if moves else 0.0)
+        # the group holding the big key: P~ = e^b (about 2^tau) against the old max, or 1 against
+        # the new one; its UOS scale byte is 127 + ceil(log2(P~max / 7.25)) either way
+        pmax = math.exp(b) if not moves else 1.0
+        assert r["p_scales"][0, T // 32] == 127 + math.ceil(math.log2(pmax / 7.25))
+        # tile 0 was quantized before any move: 64 ones, scale 2^-2 (code 6 = 4.0)
+        assert r["p_scales"][0, 0] == 125 and np.all(r["p_codes"][0, :T] == 6)
