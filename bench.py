@@ -239,9 +239,23 @@ def cpu_oracle_sample(w, target_seconds: float, causal: bool = False):
     return flops / total / 1e12, total, desc, cores
 
 
+def relaunch_ranks(n_gpus: int) -> int:
+    """`bench.py --gpus N` started without torchrun: start N ranks of this same command under
+    torch.distributed.run on this node (127.0.0.1, a free port) and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.run(cmd).returncode
+
+
 # ------------------------------------------------------------------------------------------------
 def main():
     args = parse()
+    if args.gpus > 1 and "RANK" not in os.environ:
+        sys.exit(relaunch_ranks(args.gpus))
     from mxfp4_bit_attention_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
     bf16_peak, hbm_peak, peak_kind = peaks()
@@ -258,7 +272,8 @@ def main():
                                                     args.causal)
             times.append(t)
         times = times[args.warmup:]
-        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS", "n_gpus": args.gpus,
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS",
+                "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)),
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,

@@ -306,9 +306,10 @@ MXATTN_API mxattn_status mxattn_forward(const void* q, const void* k, const void
  * mxattn_workspace_bytes_host(B, H, N, d, opts) bytes (double-buffered
  * staging and packed operands of one chunk).  Every copy and kernel is
  * ordered before the work enqueued on `stream` afterwards: synchronize
- * `stream` before reading out_host.  The call creates three non-blocking
- * streams and seven events and releases them
- * once their work completes; it allocates no memory.  Results equal
+ * `stream` before reading out_host.  The first call on a device creates
+ * three non-blocking streams and seven events for that device, kept until the
+ * process exits; calls on one device enqueue their work one at a time (a host
+ * lock).  The call allocates no device memory.  Results equal
  * mxattn_forward's bit for bit.  Errors as for mxattn_forward (a failed CUDA
  * call returns MXATTN_ERR_CUDA).  The paper has no counterpart.
  */
@@ -405,6 +406,37 @@ MXATTN_API const char* mxattn_status_string(mxattn_status status);
  * 2 * 128 * n * 64.
  */
 MXATTN_API mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream);
+
+/*
+ * Arithmetic probe (a diagnostic, not part of the method; the paper has no
+ * counterpart): evaluates one of the attention kernels' arithmetic shortcuts
+ * element-wise on n device floats `in`, writing device array `out`, so that
+ * tests can hold it against its definition.  The scale rule is opts'.
+ *   MXATTN_PROBE_EXP2_POLY            out float[n]: the FMA-pipe exp2
+ *       polynomial of the 64-key kernel at in[i]
+ *   MXATTN_PROBE_EXP2_MUFU            out float[n]: ex2.approx(in[i])
+ *   MXATTN_PROBE_E2M1_OF_EXP2_STANDIN out uint8[n]: the E2M1 code (round to
+ *       nearest even, saturating) that the 128-key kernel's FMA-pipe stand-in
+ *       for 2^u gives at u = in[i] (exact in code space by design)
+ *   MXATTN_PROBE_E2M1_OF_EXP2_MUFU    out uint8[n]: the E2M1 code of
+ *       ex2.approx(in[i])
+ *   MXATTN_PROBE_SCALE_EXP_LOG2       out int32[n]: the shared exponent e the
+ *       softmax computes for a group maximum 2^t given as t = in[i]
+ *   MXATTN_PROBE_SCALE_EXP            out int32[n]: the shared exponent e the
+ *       quantizers compute for amax = in[i] (exact integer rule)
+ * in 4-byte aligned; out 4-byte aligned for the float and int32 outputs.
+ * Invalid op, sizes or options -> MXATTN_ERR_INVALID_ARG, nothing enqueued.
+ */
+enum {
+  MXATTN_PROBE_EXP2_POLY = 0,
+  MXATTN_PROBE_EXP2_MUFU = 1,
+  MXATTN_PROBE_E2M1_OF_EXP2_STANDIN = 2,
+  MXATTN_PROBE_E2M1_OF_EXP2_MUFU = 3,
+  MXATTN_PROBE_SCALE_EXP_LOG2 = 4,
+  MXATTN_PROBE_SCALE_EXP = 5
+};
+MXATTN_API mxattn_status mxattn_arith_probe(int op, const float* in, int64_t n, const mxattn_opts* opts, void* out,
+                                            void* stream);
 
 #ifdef __cplusplus
 }

@@ -29,6 +29,7 @@ EXPORTS = (
     "mxattn_attention_mxfp4_dump", "mxattn_forward_noalloc", "mxattn_qmax_sweep",
     "mxattn_workspace_bytes_cross", "mxattn_forward_cross", "mxattn_workspace_bytes_host",
     "mxattn_forward_host", "mxattn_workspace_bytes_varlen", "mxattn_forward_varlen", "mxattn_operand_bytes",
+    "mxattn_arith_probe",
 )
 
 
@@ -104,6 +105,7 @@ def load():
         "mxattn_workspace_bytes_varlen": ([i32, i32, i32, i32, PO], sz),
         "mxattn_forward_varlen": ([P, P, P, P, i32, i32, i32, i32, f32, PO, P, P], i32),
         "mxattn_operand_bytes": ([i32, i32, i32, i32, PO, P], i32),
+        "mxattn_arith_probe": ([i32, P, i64, PO, P, P], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -394,3 +396,20 @@ def mxattn_get_device_error(workspace, stream=None) -> int:
 
 def mxattn_fp4_mma_probe(ctas: int, iters: int, n: int, stream=None):
     _check("mxattn_fp4_mma_probe", load().mxattn_fp4_mma_probe(ctas, iters, n, _stream(stream)))
+
+
+PROBE_EXP2_POLY, PROBE_EXP2_MUFU, PROBE_E2M1_STANDIN, PROBE_E2M1_MUFU, PROBE_SCALE_EXP_LOG2, PROBE_SCALE_EXP = range(6)
+
+
+def mxattn_arith_probe(op: int, x, opts: Opts | None = None, stream=None):
+    """Evaluate one of the kernels' arithmetic shortcuts on a device float32 tensor x (see the
+    header's mxattn_arith_probe); returns a device tensor (float32, uint8 or int32 by op)."""
+    import torch
+    out_dtype = {PROBE_EXP2_POLY: torch.float32, PROBE_EXP2_MUFU: torch.float32, PROBE_E2M1_STANDIN: torch.uint8,
+                 PROBE_E2M1_MUFU: torch.uint8}.get(op, torch.int32)
+    x = x.contiguous()
+    out = torch.empty(x.numel(), dtype=out_dtype, device=x.device)
+    c = _copts(opts, BF16)
+    _check("mxattn_arith_probe", load().mxattn_arith_probe(op, _ptr(x), x.numel(), ctypes.byref(c), _ptr(out),
+                                                           _stream(stream)))
+    return out

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/mxattn.h"
 #include "kernels.cuh"
@@ -505,6 +506,50 @@ mxattn_status mxattn_forward_varlen(const void* q, const void* k, const void* v,
 
 namespace {
 
+// Internal streams and events of the host-buffer forward, created once per device on first use and
+// kept until the process exits.
+struct HostStreams {
+  std::mutex mutex;  // one call at a time enqueues on them
+  cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+};
+constexpr int kMaxHostDevices = 64;
+std::mutex g_host_mutex;
+HostStreams* g_host_streams[kMaxHostDevices] = {};
+
+mxattn_status host_streams(HostStreams** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxHostDevices) return MXATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_host_mutex);
+  if (g_host_streams[dev] == nullptr) {
+    HostStreams* h = new HostStreams();
+    bool ok = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->s_c1, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->ev_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int b = 0; ok && b < 2; b++)
+      ok = cudaEventCreateWithFlags(&h->ev_in[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->ev_comp[b], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->ev_out[b], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {  // release what was made; the next call tries again
+      for (int b = 0; b < 2; b++) {
+        if (h->ev_in[b]) cudaEventDestroy(h->ev_in[b]);
+        if (h->ev_comp[b]) cudaEventDestroy(h->ev_comp[b]);
+        if (h->ev_out[b]) cudaEventDestroy(h->ev_out[b]);
+      }
+      if (h->ev_start) cudaEventDestroy(h->ev_start);
+      if (h->s_in) cudaStreamDestroy(h->s_in);
+      if (h->s_out) cudaStreamDestroy(h->s_out);
+      if (h->s_c1) cudaStreamDestroy(h->s_c1);
+      delete h;
+      return MXATTN_ERR_CUDA;
+    }
+    g_host_streams[dev] = h;
+  }
+  *out = g_host_streams[dev];
+  return MXATTN_OK;
+}
+
 // Host-buffer forward: the heads are processed in chunks, each chunk an independent problem.
 #ifndef MXATTN_HOST_CHUNKS
 #define MXATTN_HOST_CHUNKS 40
@@ -577,21 +622,23 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
   // stream and a second compute stream, each with its own operand buffers: a chunk's kernels start
   // on the SMs that the previous chunk's last wave of CTAs leaves idle instead of after it.  Every
   // cross-stream order is an event; the caller's stream finally waits for the last copies out.
-  cudaStream_t s_in = nullptr, s_out = nullptr, s_c1 = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
-  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaStreamCreateWithFlags(&s_c1, cudaStreamNonBlocking) == cudaSuccess &&
-            cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) == cudaSuccess;
-  for (int b = 0; ok && b < 2; b++)
-    ok = cudaEventCreateWithFlags(&ev_in[b], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&ev_comp[b], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&ev_out[b], cudaEventDisableTiming) == cudaSuccess;
+  // The internal streams and events are created once per device and kept; calls on one device
+  // enqueue one at a time (a host mutex), so two host threads never interleave their records.
+  HostStreams* hs = nullptr;
+  st = host_streams(&hs);
+  if (st != MXATTN_OK) return st;
+  std::lock_guard<std::mutex> lock(hs->mutex);
+  const cudaStream_t s_in = hs->s_in, s_out = hs->s_out, s_c1 = hs->s_c1;
+  cudaEvent_t const* ev_in = hs->ev_in;
+  cudaEvent_t const* ev_comp = hs->ev_comp;
+  cudaEvent_t const* ev_out = hs->ev_out;
   // work already on the caller's stream comes first
-  ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
-       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess && cudaStreamWaitEvent(s_c1, ev_start, 0) == cudaSuccess;
+  bool ok = cudaEventRecord(hs->ev_start, s) == cudaSuccess && cudaStreamWaitEvent(s_in, hs->ev_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(s_out, hs->ev_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(s_c1, hs->ev_start, 0) == cudaSuccess;
   const cudaStream_t s_comp[2] = {s, s_c1};
   st = ok ? MXATTN_OK : MXATTN_ERR_CUDA;
+  bool recorded_out[2] = {false, false};
   for (int c = 0; st == MXATTN_OK && c < p.nch; c++) {
     const int b = c & 1;
     const cudaStream_t cs = s_comp[b];  // chunk c-2 ran on it too, with the same buffers
@@ -627,22 +674,13 @@ mxattn_status mxattn_forward_host(const void* q_host, const void* k_host, const 
       st = MXATTN_ERR_CUDA;
       break;
     }
+    recorded_out[b] = true;
   }
-  // join: the caller's stream waits for every copy out (and, through them, everything else)
-  for (int b = 0; b < 2 && ev_out[b] != nullptr; b++)
-    if (cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess && st == MXATTN_OK) st = MXATTN_ERR_CUDA;
-  if (ev_start != nullptr && cudaStreamWaitEvent(s, ev_start, 0) != cudaSuccess && st == MXATTN_OK)
-    st = MXATTN_ERR_CUDA;
-  // streams and events are released once their pending work completes
-  for (int b = 0; b < 2; b++) {
-    if (ev_in[b]) cudaEventDestroy(ev_in[b]);
-    if (ev_comp[b]) cudaEventDestroy(ev_comp[b]);
-    if (ev_out[b]) cudaEventDestroy(ev_out[b]);
-  }
-  if (ev_start) cudaEventDestroy(ev_start);
-  if (s_in) cudaStreamDestroy(s_in);
-  if (s_out) cudaStreamDestroy(s_out);
-  if (s_c1) cudaStreamDestroy(s_c1);
+  // join: the caller's stream waits for every copy out of this call (and, through them, everything
+  // else), and for the internal streams' starting point
+  for (int b = 0; b < 2; b++)
+    if (recorded_out[b] && cudaStreamWaitEvent(s, ev_out[b], 0) != cudaSuccess && st == MXATTN_OK) st = MXATTN_ERR_CUDA;
+  if (cudaStreamWaitEvent(s, hs->ev_start, 0) != cudaSuccess && st == MXATTN_OK) st = MXATTN_ERR_CUDA;
   return st;
 }
 
@@ -699,6 +737,20 @@ const char* mxattn_status_string(mxattn_status s) {
     case MXATTN_ERR_TIMEOUT: return "MXATTN_ERR_TIMEOUT";
   }
   return "unknown mxattn_status";
+}
+
+mxattn_status mxattn_arith_probe(int op, const float* in, int64_t n, const mxattn_opts* o, void* out, void* stream) {
+  if (in == nullptr || out == nullptr || n < 1 || op < MXATTN_PROBE_EXP2_POLY || op > MXATTN_PROBE_SCALE_EXP)
+    return MXATTN_ERR_INVALID_ARG;
+  const mxattn_status st = check_opts(o);
+  if (st != MXATTN_OK) return st;
+  if ((reinterpret_cast<uintptr_t>(in) & 3u) != 0 || (op != MXATTN_PROBE_E2M1_OF_EXP2_STANDIN &&
+                                                      op != MXATTN_PROBE_E2M1_OF_EXP2_MUFU &&
+                                                      (reinterpret_cast<uintptr_t>(out) & 3u) != 0))
+    return MXATTN_ERR_INVALID_ARG;
+  ScaleRule r;
+  make_rule(o, &r);
+  return launched(launch_arith_probe(op, in, n, r, out, as_stream(stream)));
 }
 
 mxattn_status mxattn_fp4_mma_probe(int ctas, int iters, int n, void* stream) {

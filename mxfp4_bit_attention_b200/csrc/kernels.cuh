@@ -145,6 +145,9 @@ cudaError_t launch_qmax_sweep(const SweepArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_attention(const AttnArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_attention_wide(const AttnArgs& a, int D, int dtype, cudaStream_t s);
 cudaError_t launch_fp4_mma_probe(int ctas, int iters, int n, int* status, cudaStream_t s);
+enum { kProbeExp2Poly = 0, kProbeExp2Mufu = 1, kProbeE2m1StandIn = 2, kProbeE2m1Mufu = 3, kProbeScaleExpLog2 = 4,
+       kProbeScaleExp = 5 };
+cudaError_t launch_arith_probe(int op, const float* in, int64_t n, const ScaleRule& rule, void* out, cudaStream_t s);
 cudaError_t launch_varlen_tiles(const int* cu_seqlens, int nseq, int T, int* tile_off, int* status, cudaStream_t s);
 
 }  // namespace mxattn

@@ -66,4 +66,44 @@ cudaError_t launch_fp4_mma_probe(int ctas, int iters, int n, int* status, cudaSt
   return cudaGetLastError();
 }
 
+// Element-wise evaluation of the attention kernels' arithmetic shortcuts (device functions of
+// ptx.cuh), so that tests can hold each against its definition.  Not part of the method.
+__global__ void arith_probe_kernel(int op, const float* in, int64_t n, ScaleRule rule, void* out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const float x = in[i];
+    switch (op) {
+      case kProbeExp2Poly:
+        reinterpret_cast<float*>(out)[i] = exp2_poly2(make_float2(x, x)).x;
+        break;
+      case kProbeExp2Mufu:
+        reinterpret_cast<float*>(out)[i] = ex2_approx(x);
+        break;
+      case kProbeE2m1StandIn: {
+        const float w = fma_sat(x, 0.125f, 0.5f);  // the clamped argument the 128-key kernel feeds it
+        const float y = e2m1_exp2_stand_in(make_float2(w, w)).x;
+        reinterpret_cast<uint8_t*>(out)[i] = (uint8_t)(cvt_e2m1x8(y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xFu);
+        break;
+      }
+      case kProbeE2m1Mufu:
+        reinterpret_cast<uint8_t*>(out)[i] =
+            (uint8_t)(cvt_e2m1x8(ex2_approx(x), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xFu);
+        break;
+      case kProbeScaleExpLog2: {
+        uint32_t byte;
+        reinterpret_cast<int*>(out)[i] = (int)shared_exponent_log2f(x, rule, byte);
+        break;
+      }
+      default:  // kProbeScaleExp
+        reinterpret_cast<int*>(out)[i] = shared_exponent(x, rule);
+        break;
+    }
+  }
+}
+
+cudaError_t launch_arith_probe(int op, const float* in, int64_t n, const ScaleRule& rule, void* out, cudaStream_t s) {
+  const int64_t want = (n + 255) / 256;
+  arith_probe_kernel<<<(unsigned)(want < 4096 ? want : 4096), 256, 0, s>>>(op, in, n, rule, out);
+  return cudaGetLastError();
+}
+
 }  // namespace mxattn

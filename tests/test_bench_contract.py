@@ -57,3 +57,17 @@ def test_recorded_traffic_is_keyed_to_the_kernel_source(tmp_path, monkeypatch):
     assert b.recorded_traffic("joint") is None
     monkeypatch.setattr(b, "kernel_source_hash", lambda: "ffffffffffffffff")
     assert b.recorded_traffic("720p") is None
+
+
+def test_gpus_n_without_torchrun_starts_n_ranks():
+    """`bench.py --gpus 2` started directly (no RANK in the environment) starts two ranks under
+    torch.distributed.run on 127.0.0.1 itself; with the reference arm (no GPU needed) rank 0 prints
+    the one JSON line, reporting the world size it ran under, and the other rank exits 0."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--workload",
+           "tiny", "--steps", "1", "--warmup", "0", "--cpu-sample-seconds", "0.5"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2

@@ -100,6 +100,16 @@ def test_outlier_workload(pnq, rule, kt):
 
 
 @pytest.mark.parametrize("kt", KEY_TILES)
+def test_outlier_workload_full(kt):
+    """The outlier workload compared in full: all 4096 query rows of all 8 heads (Pith review page,
+    Fig. 4 / Proposition 1: PNQ with the UOS rule, the method's default)."""
+    w = inputs.WORKLOADS["outlier"]
+    g = inputs.generate(w)
+    got, ref = run(g, w, binding.Opts(key_tile=kt))
+    check(got, ref, f"outlier full kt={kt}")
+
+
+@pytest.mark.parametrize("kt", KEY_TILES)
 def test_output_rows_past_n_untouched(kt):
     import torch
     w = inputs.Workload("mini", 1, 2, 70, 128, "bf16", 5)

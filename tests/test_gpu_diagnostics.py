@@ -34,35 +34,66 @@ def _operands(w, g):
     return q, ops
 
 
+@pytest.mark.parametrize("kt", [64, 128])
 @pytest.mark.parametrize("name,head,qtile", [("outlier", 3, 5), ("outlier", 7, 31), ("720p", 17, 300)])
-def test_p_code_flips_against_oracle(name, head, qtile):
+def test_p_code_flips_against_oracle(name, head, qtile, kt):
     import torch
     w = inputs.WORKLOADS[name]
     g = inputs.generate(w)
     q, ops = _operands(w, g)
     scale = float(np.float32(w.d ** -0.5))
     out = torch.empty_like(q)
-    dump = binding.mxattn_attention_mxfp4_dump(ops, 1, w.H, w.N, w.d, scale, out, dump_bh=head, dump_qt=qtile)
+    dump = binding.mxattn_attention_mxfp4_dump(ops, 1, w.H, w.N, w.d, scale, out, dump_bh=head, dump_qt=qtile,
+                                               opts=binding.Opts(key_tile=kt))
     rows = np.arange(qtile * 128, min(w.N, qtile * 128 + 128))
     qf, kf, vf = (inputs.as_fp32(g[n], w.dtype)[head] for n in "qkv")
     qd, kd, vd = oracle.prepare_head(qf[rows], kf, vf)
-    ref = oracle.attention_rows(qd, kd, vd, scale, tau=8.0, codes=True)
-    T64 = (w.N + 63) // 64
+    ref = oracle.attention_rows(qd, kd, vd, scale, key_tile=kt, tau=8.0, codes=True)
+    T = (w.N + kt - 1) // kt
     n = len(rows)
-    got_codes = dump["p_codes"][:, :n, :].transpose(1, 0, 2).reshape(n, T64 * 64)[:, :w.N]
-    got_scales = dump["p_scales"][:, :n, :].transpose(1, 0, 2).reshape(n, T64 * 2)
+    got_codes = dump["p_codes"][:, :n, :].transpose(1, 0, 2).reshape(n, T * kt)[:, :w.N]
+    got_scales = dump["p_scales"][:, :n, :].transpose(1, 0, 2).reshape(n, T * (kt // 32))
     ref_codes = ref["p_codes"][:, :w.N]
     code_flips = float(np.mean(got_codes != ref_codes))
     scale_flips = float(np.mean(got_scales != ref["p_scales"]))
     # running maxima: the kernel keeps m in log2 units of the scaled scores
     m_ref = ref["m"] * np.log2(np.e)
     m_gap = float(np.max(np.abs(dump["m"][:n] - m_ref) / np.maximum(1.0, np.abs(m_ref))))
-    print("DIAG " + json.dumps({"diag": "p_code_flips", "workload": name, "head": head, "qtile": qtile,
+    print("DIAG " + json.dumps({"diag": "p_code_flips", "key_tile": kt, "workload": name, "head": head, "qtile": qtile,
                                 "rows": n, "codes": int(got_codes.size), "code_flip_fraction": code_flips,
                                 "scale_flip_fraction": scale_flips, "max_running_max_rel_gap": m_gap}))
     assert m_gap < 1e-5  # relative: the same max, up to the rounding of scale * log2(e)
     assert code_flips < 1e-3
     assert scale_flips < 1e-3
+
+
+@pytest.mark.parametrize("kt", [64, 128])
+@pytest.mark.parametrize("eps,moves", [(-1e-4, False), (1e-4, True)])
+def test_lazy_max_threshold_on_the_gpu(kt, eps, moves):
+    """The kernel's lazy running max moves only past tau = 8 in log2 units (the oracle's rule,
+    pinned on the CPU): tile 0 holds scores 0, tile 1 one key whose score is 8 (1 + eps) in log2
+    units.  Exactly representable operands (rotation off): Q rows e_0 (code 4 at scale 2^-2), the
+    key 6 e_0 (code 6 at scale 2^0); the softmax scale sets the score."""
+    import torch
+    d, N = 64, 2 * kt
+    q = np.zeros((N, d), np.float32)
+    q[:, 0] = 1.0
+    k = np.zeros((N, d), np.float32)
+    k[kt, 0] = 6.0
+    v = np.random.default_rng(3).standard_normal((N, d)).astype(np.float32)
+    scale = float(np.float32(8.0 * (1.0 + eps) * np.log(2.0) / 6.0))
+    opts = binding.Opts(rotate=False, key_tile=kt)
+    qt, kt_, vt = (torch.from_numpy(x).reshape(1, 1, N, d).cuda() for x in (q, k, v))
+    ops = binding.mxattn_quant_v(vt, opts, out=binding.mxattn_hadamard_quant_qk(qt, kt_, opts))
+    out = torch.empty_like(qt)
+    dump = binding.mxattn_attention_mxfp4_dump(ops, 1, 1, N, d, scale, out, opts=opts)
+    c = float(np.float32(scale * np.log2(np.e)))
+    expect = float(np.float32(6.0) * np.float32(c)) if moves else 0.0
+    assert np.allclose(dump["m_tiles"][0], 0.0) and np.allclose(dump["m_tiles"][1], expect, rtol=1e-6)
+    qd, kd, vd = oracle.prepare_head(q[:1], k, v, rotate=False)
+    ref = oracle.attention_rows(qd, kd, vd, scale, key_tile=kt, tau=8.0)
+    assert (ref["m"][0] > 0) == moves
+    assert np.allclose(dump["m"][:N], ref["m"][0] * np.log2(np.e), rtol=1e-6)
 
 
 def _exact_attention(q, k, v, scale):
