@@ -163,20 +163,23 @@ __device__ __forceinline__ float group_max(const uint32_t (&s)[32], int base, in
   return m[0];
 }
 
-// E2M1 codes of one group of 32: p = 2^(S*c - bias), 4 packed words.  Direct placement also
-// accumulates the unquantized p.
+// E2M1 codes of one group of 32: p = 2^((S - sm) c - e), 4 packed words.  S - sm is formed first,
+// exactly for every score near the running max (and 0 for a score equal to it), as the oracle's
+// exp(x - m) is: a score equal to the running max gives 2^-e exactly, which for e = 2 is the
+// E2M1 midpoint 0.25 that rounds to 0.  Direct placement also accumulates the unquantized p.
 template <bool MASK, bool SUM>
-__device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, int valid, float c, float bias,
-                                            uint32_t* w, float& psum) {
+__device__ __forceinline__ void group_codes(const uint32_t (&s)[32], int base, int valid, float c, float sm,
+                                            float e, uint32_t* w, float& psum) {
   const float2 cc = make_float2(c, c);
-  const float2 nb = make_float2(-bias, -bias);
+  const float2 ne = make_float2(-e, -e);
+  const float2 nsm = make_float2(-sm, -sm);
 #pragma unroll
   for (int q = 0; q < 4; q++) {
     float p[8];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      const float2 x =
-          __ffma2_rn(make_float2(__uint_as_float(s[q * 8 + i]), __uint_as_float(s[q * 8 + i + 1])), cc, nb);
+      const float2 d = __fadd2_rn(make_float2(__uint_as_float(s[q * 8 + i]), __uint_as_float(s[q * 8 + i + 1])), nsm);
+      const float2 x = __ffma2_rn(d, cc, ne);
       if (q >= 4 - kPolyWords) {
         const float2 y = exp2_poly2(x);
         p[i] = y.x;
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
       if (any_move && move) alpha = ex2_approx((sm_old - sm) * c);
 
       uint32_t eb[NG];  // scale bytes (E8M0; NVFP4: E4M3)
-      float bias[NG];
+      float bias[NG];   // MXFP4: the groups' exponents e; NVFP4: the exp2 argument's offset
       float sc[NG];     // NVFP4: the scales' values
       (void)sc;
       if constexpr (NVF) {
@@ -580,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         }
       } else {
 #pragma unroll
-        for (int g = 0; g < 2; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);
+        for (int g = 0; g < 2; g++) bias[g] = shared_exponent_log2f((gmax[g] - sm) * c, a.rule, eb[g]);  // e
       }
       uint32_t w[8];
       float psum[NG] = {};
@@ -590,11 +593,11 @@ __global__ void __launch_bounds__(kThreads, 2) mxattn_fwd_kernel(const AttnArgs 
         block16_codes<!FULL, !PNQ, false>(s1, 0, 32, valid, c, bias[2], w + 4, psum[2]);
         block16_codes<!FULL, !PNQ, true>(s1, 16, 48, valid, c, bias[3], w + 6, psum[3]);
       } else if (FULL) {
-        group_codes<false, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
-        group_codes<false, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
+        group_codes<false, !PNQ>(s0, 0, valid, c, sm, bias[0], w, psum[0]);
+        group_codes<false, !PNQ>(s1, 32, valid, c, sm, bias[1], w + 4, psum[1]);
       } else {
-        group_codes<true, !PNQ>(s0, 0, valid, c, bias[0], w, psum[0]);
-        group_codes<true, !PNQ>(s1, 32, valid, c, bias[1], w + 4, psum[1]);
+        group_codes<true, !PNQ>(s0, 0, valid, c, sm, bias[0], w, psum[0]);
+        group_codes<true, !PNQ>(s1, 32, valid, c, sm, bias[1], w + 4, psum[1]);
       }
       // test S(j+1) now, so that the test's latency overlaps the stores below
       s_ready = j + 1 < TJ && mbar_test(bar(L::B_S_FULL), (j + 1) & 1);

@@ -18,8 +18,10 @@
 //                      memory (an mbarrier per warp pair), right after the tile's max is known,
 //                      so the groups overlap everything else;
 //   warp 8 (one lane)  bulk-copies Q^ once and K^/V^ tiles + their scale atoms into a ring;
-//   warp 9             issues S = Q^ K^T (tcgen05.mma kind::mxf4 block-scaled, M128 N128);
-//   warp 10            issues O~ += P^ V^ (two K = 64 MMAs per tile, M128 N = d + 16).
+//   warps 9, 10        issue S = Q^ K^T (tcgen05.mma kind::mxf4 block-scaled, M128 N128) for the
+//                      tiles of softmax group 0 and 1 respectively, so that neither group's next
+//                      S waits behind the other's buffer release;
+//   warp 11            issues O~ += P^ V^ (two K = 64 MMAs per tile, M128 N = d + 16).
 // P^ is written in four shared-memory buffers (two per group), so the softmax never waits for
 // the PV MMA of its own previous tile.  PNQ row sum: V^'s operand image carries 16 extra rows
 // after its d channel rows, the first all ones (scale 2^0), so the PV MMA also accumulates
@@ -45,8 +47,8 @@ constexpr int kBN = 128;   // keys per tile
 enum { kModeFull = 0, kModeDump = 1, kModeMasked = 2 };
 constexpr int kStages = 5;  // K/V shared-memory ring depth
 constexpr int kPBufs = 4;   // P^ buffers (tile j uses j % 4)
-constexpr int kProducerWarp = 8, kQkWarp = 9, kPvWarp = 10;
-constexpr int kWarps = 11;
+constexpr int kProducerWarp = 8, kQkWarp = 9, kPvWarp = 11;  // warps 9 and 10 issue QK for groups 0 and 1
+constexpr int kWarps = 12;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kOnesRows = 16;  // rows appended to each 64-key half of V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 512;
@@ -60,7 +62,7 @@ constexpr uint32_t kPolyMask = MXATTN_WIDE_POLY_MASK;
 
 template <int D>
 struct Layout {
-  static constexpr int K_SLOTS = 3;  // K scale-factor slots in TMEM (slot j % 3)
+  static constexpr int K_SLOTS = 4;  // K scale-factor slots in TMEM: two per QK issuer
   static constexpr int V_SLOTS = 5;  // V scale-factor slots in TMEM (slot j % 5)
   // shared memory, byte offsets from a 1024-byte aligned base
   static constexpr int Q_BYTES = kBM * D / 2;
@@ -105,8 +107,8 @@ struct Layout {
   // tensor memory columns
   static constexpr uint32_t T_S = 0;                  // S buffers: group g at 128 g
   static constexpr uint32_t T_O = 256;                // O~: D columns, then l at column D
-  static constexpr uint32_t T_SFQ = T_O + D + kOnesRows;
-  static constexpr uint32_t T_SFP = T_SFQ + 4;        // kPBufs x 4 columns
+  static constexpr uint32_t T_SFQ = T_O + D + kOnesRows;  // Q scales, one copy per QK issuer
+  static constexpr uint32_t T_SFP = T_SFQ + 8;        // kPBufs x 4 columns
   static constexpr uint32_t T_SFK = T_SFP + 4 * kPBufs;  // K_SLOTS x 4 columns
   static constexpr uint32_t T_SFV = T_SFK + 4 * K_SLOTS; // V_SLOTS x 8 columns (V atom + ones atom)
   static_assert(T_SFV + 8 * V_SLOTS <= kTmemCols, "TMEM budget");
@@ -118,34 +120,43 @@ __device__ __forceinline__ void raise_abort(volatile int* flag, int* status, int
   if (atomicCAS(status, 0, kStatusTimeout) == 0) atomicExch(status + 1, where);
 }
 
-// maximum of 32 raw S values, two independent chains of three-input maxima
-__device__ __forceinline__ float max32(const uint32_t* s) {
-  float a = -INFINITY, b = -INFINITY;
+// Maxima of the four 32-key groups of a 128-key tile, eight independent chains of three-input
+// maxima advanced together so that their latencies overlap.
+__device__ __forceinline__ void group_maxima(const uint32_t (&s)[128], float (&gmax)[4]) {
+  float a[4], b[4];
+#pragma unroll
+  for (int g = 0; g < 4; g++) a[g] = b[g] = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 32; i += 4) {
-    a = fmax3(a, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-    b = fmax3(b, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+#pragma unroll
+    for (int g = 0; g < 4; g++) {
+      a[g] = fmax3(a[g], __uint_as_float(s[32 * g + i]), __uint_as_float(s[32 * g + i + 1]));
+      b[g] = fmax3(b[g], __uint_as_float(s[32 * g + i + 2]), __uint_as_float(s[32 * g + i + 3]));
+    }
   }
-  return fmaxf(a, b);
+#pragma unroll
+  for (int g = 0; g < 4; g++) gmax[g] = fmaxf(a[g], b[g]);
 }
 
-// E2M1 codes of one 8-key word, p = 2^(S c - bias): MUFU ex2, or (POLY) the FMA-pipe stand-in fed
-// with w = clamp((S c - bias + 4) / 8, 0, 1) = sat(S cs + bs).  SUM: direct placement, also
-// accumulates the unquantized p.
+// E2M1 codes of one 8-key word, p = 2^((S - sm) c - e).  S - sm is formed first, exactly for every
+// score near the running max (and 0 for a score equal to it), as the oracle's exp(x - m) is, so a
+// score equal to the running max gives 2^-e exactly (for e = 2 the E2M1 midpoint 0.25, which
+// rounds to 0).  MUFU ex2, or (POLY) the FMA-pipe stand-in fed with
+// w = clamp(((S - sm) c - e + 2.5) / 8, 0, 1) = sat((S - sm) cs + bs).  SUM: direct placement,
+// also accumulates the unquantized p.
 template <bool POLY, bool SUM>
-__device__ __forceinline__ uint32_t word_codes(const uint32_t* s, float c, float nbias, float cs, float bs,
+__device__ __forceinline__ uint32_t word_codes(const uint32_t* s, float sm, float c, float e, float cs, float bs,
                                                float& psum) {
   float p[8];
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
+    const float2 d = __fadd2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), make_float2(-sm, -sm));
     if (POLY) {
-      const float2 w = make_float2(fma_sat(__uint_as_float(s[i]), cs, bs), fma_sat(__uint_as_float(s[i + 1]), cs, bs));
-      const float2 y = e2m1_exp2_stand_in(w);
+      const float2 y = e2m1_exp2_stand_in(make_float2(fma_sat(d.x, cs, bs), fma_sat(d.y, cs, bs)));
       p[i] = y.x;
       p[i + 1] = y.y;
     } else {
-      const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), make_float2(c, c),
-                                  make_float2(nbias, nbias));
+      const float2 x = __ffma2_rn(d, make_float2(c, c), make_float2(-e, -e));
       p[i] = ex2_approx(x.x);
       p[i + 1] = ex2_approx(x.y);
       if (SUM) psum += p[i] + p[i + 1];
@@ -156,18 +167,17 @@ __device__ __forceinline__ uint32_t word_codes(const uint32_t* s, float c, float
 
 // the four words of 32-key group G (words 4G..4G+3 of the tile)
 template <int G, bool PNQ>
-__device__ __forceinline__ void group_codes(const uint32_t (&s)[128], float c, float bias, uint32_t* w,
+__device__ __forceinline__ void group_codes(const uint32_t (&s)[128], float sm, float c, float e, uint32_t* w,
                                             float& psum) {
-  const float nbias = -bias;
   const float cs = c * 0.125f;
-  const float bs = __fmaf_rn(bias, -0.125f, 0.5f);
+  const float bs = (-kStandInLo - e) * 0.125f;  // exact: e is a small integer
 #pragma unroll
   for (int q = 0; q < 4; q++) {
     constexpr uint32_t mask = PNQ ? kPolyMask : 0u;
     if ((mask >> (4 * G + q)) & 1u)
-      w[q] = word_codes<true, false>(s + 32 * G + 8 * q, c, nbias, cs, bs, psum);
+      w[q] = word_codes<true, false>(s + 32 * G + 8 * q, sm, c, e, cs, bs, psum);
     else
-      w[q] = word_codes<false, !PNQ>(s + 32 * G + 8 * q, c, nbias, cs, bs, psum);
+      w[q] = word_codes<false, !PNQ>(s + 32 * G + 8 * q, sm, c, e, cs, bs, psum);
   }
 }
 
@@ -240,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     }
     for (int i = 0; i < 8; i++) mbar_init(bar(L::B_XCH + i), 1);
     mbar_init(bar(L::B_EPI), 8);
-    mbar_init(bar(L::B_DRAIN), 2);  // one commit from each issuer
+    mbar_init(bar(L::B_DRAIN), 3);  // one commit from each issuer
     fence_mbar_init();
   }
   if (PNQ) {
@@ -301,24 +311,27 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; j++)
         mbar_wait(bar(L::B_KV_FULL + j % kStages), (j / kStages) & 1, no_abort, kDrainBudgetCycles);
     }
-  } else if (warp == kQkWarp) {
-    // ------------------------------------------------------------------ QK issuer
-    // The warp runs the loop converged (waits and descriptor arithmetic stay warp-uniform); lane 0
-    // alone issues its tcgen05 operations, so that each of its commits covers all of them.
+  } else if (warp == kQkWarp || warp == kQkWarp + 1) {
+    // ------------------------------------------------------------------ QK issuers
+    // Issuer g serves the tiles of softmax group g.  The warp runs the loop converged (waits and
+    // descriptor arithmetic stay warp-uniform); lane 0 alone issues its tcgen05 operations, so that
+    // each of its commits covers all of them.
+    const int g = warp - kQkWarp;
     const bool leader = lane == 0;
+    const uint32_t t_sfq = tmem + L::T_SFQ + 4 * g;  // this issuer's own copy of the Q scales
     bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget));
     if (ok) {
       tc_fence_after();
-      if (leader) tmem_cp_sf_atom(tmem + L::T_SFQ, sb + L::SF_Q);
+      if (leader) tmem_cp_sf_atom(t_sfq, sb + L::SF_Q);
       __syncwarp();
       const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
-      for (int j = 0; j < TJ; j++) {
-        const int s = j % kStages, f = j % L::K_SLOTS, g = j & 1;
+      for (int j = g; j < TJ; j += 2) {
+        const int s = j % kStages, f = 2 * g + ((j >> 1) & 1);
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
         if (!ok) break;
         tc_fence_after();
-        // K scale slot f was last read by QK(j-3), complete since group (j-3)&1 read that S before
-        // releasing it, which this warp waited for before issuing QK(j-1)
+        // K scale slot f was last read by QK(j-4), complete since group g read that S before
+        // releasing it, which this warp waited for before issuing QK(j-2)
         if (leader) tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
         if (j >= 2) {  // S buffer g was last read by group g at tile j-2
           ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_S_FREE + g), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget));
@@ -330,11 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
 #pragma unroll
           for (int kb = 0; kb < D / 64; kb++)  // head dims 64kb..: 32 bytes along each row, scale bytes 2kb, 2kb+1
             mma_mxf4(tmem + L::T_S + 128 * g, qdesc + (uint64_t)(kb * 2), kdesc + (uint64_t)(kb * 2),
-                     mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), tmem + L::T_SFQ, tmem + L::T_SFK + 4 * f, kb > 0 ? 1u : 0u);
+                     mxf4_idesc(kBM, kBN, 2 * kb, 2 * kb), t_sfq, tmem + L::T_SFK + 4 * f, kb > 0 ? 1u : 0u);
         }
         if (j >= kPBufs) {
           // S(j) also tells group g that P buffer j % 4 (last read by PV(j-4)) is free: see PV(j-4)
-          // complete before committing S(j).  Each O_DONE barrier is at most one phase away here.
+          // complete before committing S(j).  Each O_DONE barrier is at most one phase away here:
+          // PV(j) needs S(j), and this issuer saw PV(j-8) complete before committing S(j-4).
           const int pb = j % kPBufs;
           ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + pb), ((j - kPBufs) / kPBufs) & 1, abort_flag,
                                                  a.wait_budget));
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       }
     }
     if (!ok && leader) raise_abort(abort_flag, a.status, 2);
-    // wait for every tcgen05 operation of both issuers before TMEM is released
+    // wait for every tcgen05 operation of the three issuers before TMEM is released
     if (leader) mma_commit(bar(L::B_DRAIN));
     __syncwarp();
     mbar_wait(bar(L::B_DRAIN), 0, no_abort, kDrainBudgetCycles);
@@ -421,8 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         if (!__all_sync(0xFFFFFFFFu, ok)) return false;
       }
       tc_fence_after();
+      const uint32_t sbuf = tl + L::T_S + 128 * grp;
       uint32_t s[128];
-      tmem_ld128_wait(tl + L::T_S + 128 * grp, s);
+      tmem_ld128_wait(sbuf, s);
+      // S(j) is in registers: the QK MMA of tile j+2 may overwrite the buffer
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::B_S_FREE + grp));
@@ -437,8 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         for (int i = 0; i < 128; i++) ds[i] = __uint_as_float(s[i]);
       }
       float gmax[4];
-#pragma unroll
-      for (int g = 0; g < 4; g++) gmax[g] = max32(s + 32 * g);
+      group_maxima(s, gmax);
       const float mt_raw = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3]));
       // the running max after tile j-1, handed over by the other group
       float sm_prev = -INFINITY;
@@ -467,15 +482,19 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       sm = sm_new;
 
       uint32_t eb[4];
-      float bias[4];
+      float ex[4];  // the groups' shared exponents e
 #pragma unroll
-      for (int g = 0; g < 4; g++) bias[g] = m2 + shared_exponent_log2f((gmax[g] - sm_new) * c, a.rule, eb[g]);
+      for (int g = 0; g < 4; g++) ex[g] = shared_exponent_log2f((gmax[g] - sm_new) * c, a.rule, eb[g]);
       uint32_t w[16];
       float psum[4] = {0.f, 0.f, 0.f, 0.f};
-      group_codes<0, PNQ>(s, c, bias[0], w, psum[0]);
-      group_codes<1, PNQ>(s, c, bias[1], w + 4, psum[1]);
-      group_codes<2, PNQ>(s, c, bias[2], w + 8, psum[2]);
-      group_codes<3, PNQ>(s, c, bias[3], w + 12, psum[3]);
+      group_codes<0, PNQ>(s, sm_new, c, ex[0], w, psum[0]);
+      group_codes<1, PNQ>(s, sm_new, c, ex[1], w + 4, psum[1]);
+      group_codes<2, PNQ>(s, sm_new, c, ex[2], w + 8, psum[2]);
+      group_codes<3, PNQ>(s, sm_new, c, ex[3], w + 12, psum[3]);
+      if (dumping) {  // the unquantized tile, relative to this tile's running max
+        float* dpt = reinterpret_cast<float*>(a.dump + dl.p_tilde) + ((size_t)j * 128 + row) * kBN;
+        for (int i = 0; i < 128; i++) dpt[i] = ex2_approx((__uint_as_float(s[i]) - sm_new) * c);
+      }
       // test S(j+2) now, so that the test's latency overlaps the stores below
       s_ready = j + 2 < TJ && mbar_test(bar(L::B_S_FULL + grp), ((j + 2) >> 1) & 1);
       if (!PNQ) {
@@ -528,8 +547,6 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         uint8_t* dsf = a.dump + dl.p_scales + ((size_t)j * 128 + row) * 4;
         for (int g = 0; g < 4; g++) dsf[g] = (uint8_t)eb[g];
         // the unquantized tile, relative to this tile's running max (dump only)
-        float* dpt = reinterpret_cast<float*>(a.dump + dl.p_tilde) + ((size_t)j * 128 + row) * kBN;
-        for (int i = 0; i < 128; i++) dpt[i] = ex2_approx(__fmaf_rn(__uint_as_float(s[i]), c, -m2));
         reinterpret_cast<float*>(a.dump + dl.m_tiles)[(size_t)j * 128 + row] = m2;
       }
       return true;

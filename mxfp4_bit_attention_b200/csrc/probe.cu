@@ -79,7 +79,7 @@ __global__ void arith_probe_kernel(int op, const float* in, int64_t n, ScaleRule
         reinterpret_cast<float*>(out)[i] = ex2_approx(x);
         break;
       case kProbeE2m1StandIn: {
-        const float w = fma_sat(x, 0.125f, 0.5f);  // the clamped argument the 128-key kernel feeds it
+        const float w = fma_sat(x, 0.125f, -kStandInLo * 0.125f);  // the clamped argument the 128-key kernel feeds it
         const float y = e2m1_exp2_stand_in(make_float2(w, w)).x;
         reinterpret_cast<uint8_t*>(out)[i] = (uint8_t)(cvt_e2m1x8(y, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f) & 0xFu);
         break;

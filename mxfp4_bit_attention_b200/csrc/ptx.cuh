@@ -400,10 +400,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // 2^x for a pair of fp32 values on the FMA pipe (no MUFU): Cody-Waite style range reduction
 // x = n + f, n = round(x) via the 1.5 * 2^23 rounding constant, f in [-0.5, 0.5]; 2^f by a
-// degree-5 polynomial (our own minimax fit of 2^f on [-0.5, 0.5], relative error 7.5e-8 before
-// fp32 rounding, 2.2e-7 measured with fp32 Horner evaluation); 2^n added to the exponent
-// field.  Inputs are clamped below at -64 (2^-64 is far below every rounding threshold that
-// matters here); inputs are at most a few units above 0 in the attention kernel.
+// degree-5 polynomial with constant term exactly 1 (our own fit of 2^f on [-0.5, 0.5] by
+// reweighted least squares toward minimax relative error, 1.9e-7 with fp32 Horner evaluation),
+// so that integer x gives 2^x exactly; 2^n added to the exponent field.  Inputs are clamped below
+// at -64 (2^-64 is far below every rounding threshold that matters here); inputs are at most a
+// few units above 0 in the attention kernel.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   x.x = fmaxf(x.x, -64.f);
@@ -411,11 +412,11 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));                         // kRound + n
   const float2 nn = __ffma2_rn(t, make_float2(-1.f, -1.f), make_float2(kRound, kRound));  // -n
   const float2 f = __fadd2_rn(x, nn);                                                  // x - n
-  float2 p = __ffma2_rn(make_float2(1.3276472e-3f, 1.3276472e-3f), f, make_float2(9.6755410e-3f, 9.6755410e-3f));
-  p = __ffma2_rn(p, f, make_float2(5.5507131e-2f, 5.5507131e-2f));
-  p = __ffma2_rn(p, f, make_float2(2.4022120e-1f, 2.4022120e-1f));
-  p = __ffma2_rn(p, f, make_float2(6.9314694e-1f, 6.9314694e-1f));
-  p = __ffma2_rn(p, f, make_float2(1.0000001f, 1.0000001f));
+  float2 p = __ffma2_rn(make_float2(1.3264724e-3f, 1.3264724e-3f), f, make_float2(9.6715130e-3f, 9.6715130e-3f));
+  p = __ffma2_rn(p, f, make_float2(5.5507336e-2f, 5.5507336e-2f));
+  p = __ffma2_rn(p, f, make_float2(2.4022242e-1f, 2.4022242e-1f));
+  p = __ffma2_rn(p, f, make_float2(6.9314700e-1f, 6.9314700e-1f));
+  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
   // the low bits of t hold n; (bits(t) << 23) adds n to the exponent (the constant's own bits
   // shift out entirely)
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
@@ -435,45 +436,33 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   return d;
 }
 
-// bits(q) + bits(t) * 2^23 in one integer multiply-add: adds the integer held in the low bits of
-// t to q's exponent field.
-__device__ __forceinline__ float add_exponent(float q, float t) {
-  uint32_t r;
-  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r) : "r"(__float_as_uint(t)), "r"(__float_as_uint(q)));
-  return __uint_as_float(r);
-}
-
 // A stand-in for 2^u that gives the same E2M1 code as 2^u under cvt.rn.satfinite.e2m1x2 (round to
-// nearest even, saturating at 6), for a pair of arguments given as w = clamp((u + 4) / 8, 0, 1),
-// computed on the FMA pipe alone.
+// nearest even, saturating at 6), for a pair of arguments given as w = clamp((u + 2.5) / 8, 0, 1),
+// computed on the FMA pipe alone with six packed FMAs.
 //
 // The E2M1 code of a positive value depends only on where it lies against the grid midpoints
-// 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5.  Writing u = k + f (k = floor u, f in [0, 1)), every
-// midpoint is 2^k times one of 1 (k = -2: the 0.25 tie, which rounds to 0), 1.25, 1.5 (k = -1:
-// 0.75) or 1.75.  So the value 2^k * q(f) gets the code of 2^u whenever q is increasing on [0, 1),
-// meets 2^f at f = log2 1.25, log2 1.5 and log2 1.75, stays above 1 at f = 0 and below 2 as f -> 1
-// (then the step at each integer k crosses 0.25 only at u = -2 exactly and crosses no other
-// midpoint).  The quadratic through those three points does all of this: q(0) = 1.0114,
-// q(1) = 1.9952, q' > 0.  Arguments below -4 map to k = -4 (2^-4 * q < 0.25: code 0); the
-// clamp also keeps k in a range where adding it to the exponent field cannot wrap.  The result
-// is a code-exact stand-in, not an accurate exponential: use it only in front of the E2M1
-// conversion.
-constexpr float kQuadC0 = 1.0114069778f;
-constexpr float kQuadC1 = 0.6259469002f;
-constexpr float kQuadC2 = 0.3578150505f;
-constexpr float kFloorMagic = 12582912.f;  // 1.5 * 2^23: integers in the low mantissa bits
+// 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5, i.e. on where u lies against their base-2 logarithms.
+// So any function P of w that is increasing on [0, 1] and takes the midpoint values at those seven
+// arguments gives every u its code (P(0) = 0.19 < 0.25: code 0 below the range; P(1) = 43 > 5:
+// code 7 above it).  P is the degree-6 polynomial through the seven points (monotone on [0, 1],
+// checked on a dense grid), with one change: at u = -2 it takes 0.25 (1 - 2^-20) instead of 0.25,
+// so that u = -2 exactly (a score equal to the running max in a group of scale 2^2, whose
+// exponential is exactly the tie 0.25 and rounds to 0) stays below the tie whatever the rounding
+// of the evaluation; only u within 1.4e-6 above -2 is given code 0 instead of 1 by this.  Every
+// other integer u lands on a grid value, far from any midpoint.  The result is a code-exact
+// stand-in, not an accurate exponential: use it only in front of the E2M1 conversion.
+constexpr float kStandInLo = -2.5f;   // w = (u - kStandInLo) / 8
+constexpr float kStandInC0 = 0.19134787f, kStandInC1 = 0.54114223f, kStandInC2 = 7.1855769f,
+                kStandInC3 = -17.132305f, kStandInC4 = 66.555229f, kStandInC5 = -78.487640f,
+                kStandInC6 = 64.299675f;
 
 __device__ __forceinline__ float2 e2m1_exp2_stand_in(float2 w) {
-  const float2 m4 = make_float2(kFloorMagic - 4.f, kFloorMagic - 4.f);
-  const float2 eight = make_float2(8.f, 8.f);
-  // t = M + floor(8w - 4): the sum is positive, so rounding toward zero is rounding down
-  const float2 t = __ffma2_rz(w, eight, m4);
-  const float2 nk = __ffma2_rn(t, make_float2(-1.f, -1.f), m4);  // -floor(8w), exact
-  const float2 f = __ffma2_rn(w, eight, nk);                       // 8w - floor(8w), exact
-  float2 q = __ffma2_rn(f, make_float2(kQuadC2, kQuadC2), make_float2(kQuadC1, kQuadC1));
-  q = __ffma2_rn(q, f, make_float2(kQuadC0, kQuadC0));
-  // the low bits of t hold k (the constant's own bits shift out of the 32-bit product)
-  return make_float2(add_exponent(q.x, t.x), add_exponent(q.y, t.y));
+  float2 p = __ffma2_rn(w, make_float2(kStandInC6, kStandInC6), make_float2(kStandInC5, kStandInC5));
+  p = __ffma2_rn(p, w, make_float2(kStandInC4, kStandInC4));
+  p = __ffma2_rn(p, w, make_float2(kStandInC3, kStandInC3));
+  p = __ffma2_rn(p, w, make_float2(kStandInC2, kStandInC2));
+  p = __ffma2_rn(p, w, make_float2(kStandInC1, kStandInC1));
+  return __ffma2_rn(p, w, make_float2(kStandInC0, kStandInC0));
 }
 
 __device__ __forceinline__ float lg2_approx(float x) {

@@ -249,97 +249,132 @@ __global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
 
 // ------------------------------------------------------------------------------------------------
 // V: quantization along keys (32 consecutive tokens per channel) into the packed V operand
-// layout.  One block per (head, 64-key tile): the tile is staged through shared memory as
-// fp32 [64][D+1], then thread (channel c, half h) quantizes keys 32h..32h+31 of channel c.
-// Varlen: blocks over (head, 64-key tile of the packed tiles); each sequence's groups start at
-// its first token, and a sequence's tiles past its own keys are left unwritten.
+// layout.  Blocks stride over the (head, 64-key tile) items; each tile is staged through shared
+// memory as fp32 [64][D+1], then thread (channel c, half h) quantizes keys 32h..32h+31 of channel
+// c.  The next tile's inputs are loaded into registers before the current tile is quantized, so
+// a load is always in flight while the block computes.
+// Varlen: items over (head, 64-key tile of the packed tiles); each sequence's groups start at its
+// first token, and a sequence's tiles past its own keys are left unwritten.
 // ------------------------------------------------------------------------------------------------
-template <int D, int DT, bool NVF>
-__global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a) {
-  __shared__ float tile[64][D + 1];
-  const bool vl = a.vl.cu_seqlens != nullptr;
-  int N = a.N;                                  // keys of this block's sequence
-  int T64, bh, j;                               // its 64-key tiles, head, and this tile among them
-  int64_t src_row0, src_stride;                 // source row of key 0 and the row step per key
-  int64_t vtile, atom_tile;                     // packed 64-key code tile and 128-key scale atom
-  if (vl) {
+struct VTile {
+  bool ok;                 // the item holds keys of a sequence
+  int N, T64, j;           // keys of its sequence, their 64-key tiles, and this tile among them
+  int64_t src_row0;        // source row of key 0
+  int64_t src_stride;      // source rows per key
+  int64_t vtile;           // packed 64-key code tile
+  int64_t atom_tile;       // packed 128-key scale atom
+};
+
+__device__ __forceinline__ VTile v_tile(const VQuantArgs& a, int64_t item) {
+  VTile t;
+  t.ok = true;
+  if (a.vl.cu_seqlens != nullptr) {
     const int per_head = 2 * a.vl.tiles_per_head;
-    bh = blockIdx.x / per_head;
-    const int jg = blockIdx.x % per_head;
-    if (jg / 2 >= __ldg(a.vl.tile_off + a.vl.nseq)) return;
+    const int bh = (int)(item / per_head);
+    const int jg = (int)(item % per_head);
+    if (jg / 2 >= __ldg(a.vl.tile_off + a.vl.nseq)) {
+      t.ok = false;
+      return t;
+    }
     const int sq = varlen_sequence(a.vl, jg / 2);
     const int start = __ldg(a.vl.cu_seqlens + sq);
-    N = __ldg(a.vl.cu_seqlens + sq + 1) - start;
-    T64 = (N + 63) / 64;
-    j = jg - 2 * __ldg(a.vl.tile_off + sq);
-    if (j >= T64) return;                       // the unused odd half of a sequence's last atom
-    src_row0 = (int64_t)start * a.BH + bh;
-    src_stride = a.BH;
-    vtile = (int64_t)bh * per_head + jg;
-    atom_tile = (int64_t)bh * a.vl.tiles_per_head + jg / 2;
+    t.N = __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    t.T64 = (t.N + 63) / 64;
+    t.j = jg - 2 * __ldg(a.vl.tile_off + sq);
+    t.ok = t.j < t.T64;  // not the unused odd half of a sequence's last atom
+    t.src_row0 = (int64_t)start * a.BH + bh;
+    t.src_stride = a.BH;
+    t.vtile = (int64_t)bh * per_head + jg;
+    t.atom_tile = (int64_t)bh * a.vl.tiles_per_head + jg / 2;
   } else {
-    T64 = (N + 63) / 64;
-    bh = blockIdx.x / T64;
-    j = blockIdx.x % T64;
-    src_row0 = (int64_t)bh * N;
-    src_stride = 1;
-    vtile = (int64_t)bh * T64 + j;
-    atom_tile = (int64_t)bh * ((N + 127) / 128) + j / 2;
+    t.N = a.N;
+    t.T64 = (a.N + 63) / 64;
+    const int bh = (int)(item / t.T64);
+    t.j = (int)(item % t.T64);
+    t.src_row0 = (int64_t)bh * a.N;
+    t.src_stride = 1;
+    t.vtile = item;
+    t.atom_tile = (int64_t)bh * ((a.N + 127) / 128) + t.j / 2;
   }
+  return t;
+}
+
+template <int D, int DT, bool NVF>
+__global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a, int64_t items) {
+  __shared__ float tile[64][D + 1];
+  constexpr int VEC_PER_ROW = D / 8;             // 8 values per load
+  constexpr int NVEC = 64 * VEC_PER_ROW / 256;   // loads per thread and tile
   const int t = threadIdx.x;
-  // stage: 64 tokens x D values, 8 values per thread-iteration
-  constexpr int VEC_PER_ROW = D / 8;
-  // a fixed trip count (64 * D / 8 / 256): unrolled, so every thread has all its loads in flight
+  float nxt[NVEC][8];
+  auto load_tile = [&](const VTile& vt) {
 #pragma unroll
-  for (int idx = t; idx < 64 * VEC_PER_ROW; idx += 256) {
-    const int row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
-    const int tok = j * 64 + row;
-    float v[8];
-    load8<DT>(a.v, (src_row0 + (tok < N ? tok : 0) * src_stride) * D + cv * 8, tok < N, v);
+    for (int u = 0; u < NVEC; u++) {
+      const int idx = t + 256 * u, row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
+      const int tok = vt.j * 64 + row;
+      const bool valid = vt.ok && tok < vt.N;
+      load8<DT>(a.v, (vt.src_row0 + (valid ? tok : 0) * vt.src_stride) * D + cv * 8, valid, nxt[u]);
+    }
+  };
+  int64_t item = blockIdx.x;
+  VTile next = v_tile(a, item);
+  load_tile(next);
+  for (; item < items; item += gridDim.x) {
+    __syncthreads();  // the previous tile has been read out of shared memory
 #pragma unroll
-    for (int i = 0; i < 8; i++) tile[row][cv * 8 + i] = v[i];
-  }
-  __syncthreads();
-  for (int item = t; item < 2 * D; item += 256) {
-    const int c = item % D, h = item / D;
-    if (NVF) {
-      // two blocks of 16 keys; one scale atom per 64-key tile, keys 16b..16b+15 in byte b of
-      // channel c's word
-      float x[32];
+    for (int u = 0; u < NVEC; u++) {
+      const int idx = t + 256 * u, row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
 #pragma unroll
-      for (int i = 0; i < 32; i++) x[i] = tile[h * 32 + i][c];
+      for (int i = 0; i < 8; i++) tile[row][cv * 8 + i] = nxt[u][i];
+    }
+    const VTile me = next;
+    if (item + gridDim.x < items) {
+      next = v_tile(a, item + gridDim.x);
+      load_tile(next);  // in flight while this tile is quantized
+    }
+    __syncthreads();
+    if (!me.ok) continue;
+    const int j = me.j;
+    for (int it = t; it < 2 * D; it += 256) {
+      const int c = it % D, h = it / D;
+      if (NVF) {
+        // two blocks of 16 keys; one scale atom per 64-key tile, keys 16b..16b+15 in byte b of
+        // channel c's word
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) x[i] = tile[h * 32 + i][c];
+        uint32_t w[4];
+        const uint32_t b = nvfp4_block(x, w) | (nvfp4_block(x + 16, w + 2) << 8);
+        uint8_t* dst = a.v_codes + (me.vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        uint8_t* atom = a.v_scales + me.vtile * 512;
+        *reinterpret_cast<uint16_t*>(atom + (c % 32) * 16 + (c / 32) * 4 + 2 * h) = (uint16_t)b;
+        if (D == 64) *reinterpret_cast<uint16_t*>(atom + ((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 * h) = 0;
+        continue;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(tile[h * 32 + i][c]));
+      const int e = shared_exponent(amax, a.rule);
+      const float inv = pow2_neg(e);
       uint32_t w[4];
-      const uint32_t b = nvfp4_block(x, w) | (nvfp4_block(x + 16, w + 2) << 8);
-      uint8_t* dst = a.v_codes + (vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const int b = h * 32 + q * 8;
+        w[q] = cvt_e2m1x8(__fmul_rn(tile[b + 0][c], inv), __fmul_rn(tile[b + 1][c], inv),
+                          __fmul_rn(tile[b + 2][c], inv), __fmul_rn(tile[b + 3][c], inv),
+                          __fmul_rn(tile[b + 4][c], inv), __fmul_rn(tile[b + 5][c], inv),
+                          __fmul_rn(tile[b + 6][c], inv), __fmul_rn(tile[b + 7][c], inv));
+      }
+      uint8_t* dst = a.v_codes + (me.vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-      uint8_t* atom = a.v_scales + vtile * 512;
-      *reinterpret_cast<uint16_t*>(atom + (c % 32) * 16 + (c / 32) * 4 + 2 * h) = (uint16_t)b;
-      if (D == 64) *reinterpret_cast<uint16_t*>(atom + ((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 * h) = 0;
-      continue;
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(tile[h * 32 + i][c]));
-    const int e = shared_exponent(amax, a.rule);
-    const float inv = pow2_neg(e);
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const int b = h * 32 + q * 8;
-      w[q] = cvt_e2m1x8(__fmul_rn(tile[b + 0][c], inv), __fmul_rn(tile[b + 1][c], inv),
-                        __fmul_rn(tile[b + 2][c], inv), __fmul_rn(tile[b + 3][c], inv),
-                        __fmul_rn(tile[b + 4][c], inv), __fmul_rn(tile[b + 5][c], inv),
-                        __fmul_rn(tile[b + 6][c], inv), __fmul_rn(tile[b + 7][c], inv));
-    }
-    uint8_t* dst = a.v_codes + (vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    uint8_t* atom = a.v_scales + atom_tile * 512;
-    atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
-    if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
-    // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
-    if (j == T64 - 1 && (j % 2) == 0) {
-      atom[(c % 32) * 16 + (c / 32) * 4 + 2 + h] = 0;
-      if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 + h] = 0;
+      uint8_t* atom = a.v_scales + me.atom_tile * 512;
+      atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
+      if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
+      // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
+      if (j == me.T64 - 1 && (j % 2) == 0) {
+        atom[(c % 32) * 16 + (c / 32) * 4 + 2 + h] = 0;
+        if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 + h] = 0;
+      }
     }
   }
 }
@@ -420,14 +455,17 @@ cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaS
 }
 
 template <int D, int DT>
-static void v_launch(const VQuantArgs& a, unsigned blocks, cudaStream_t s) {
-  if (a.fmt == kFmtNVFP4) quant_v_kernel<D, DT, true><<<blocks, 256, 0, s>>>(a);
-  else quant_v_kernel<D, DT, false><<<blocks, 256, 0, s>>>(a);
+static void v_launch(const VQuantArgs& a, int64_t items, cudaStream_t s) {
+  // several blocks per SM (33 KB of shared memory each at D = 128), each striding over the items
+  constexpr int64_t kMaxBlocks = 148 * 6;
+  const unsigned blocks = (unsigned)(items < kMaxBlocks ? items : kMaxBlocks);
+  if (a.fmt == kFmtNVFP4) quant_v_kernel<D, DT, true><<<blocks, 256, 0, s>>>(a, items);
+  else quant_v_kernel<D, DT, false><<<blocks, 256, 0, s>>>(a, items);
 }
 
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s) {
-  const unsigned blocks = (unsigned)((int64_t)a.BH * (a.vl.cu_seqlens != nullptr ? 2 * (int64_t)a.vl.tiles_per_head
-                                                                                 : (a.N + 63) / 64));
+  const int64_t blocks = (int64_t)a.BH * (a.vl.cu_seqlens != nullptr ? 2 * (int64_t)a.vl.tiles_per_head
+                                                                     : (a.N + 63) / 64);
   if (D == 128 && dtype == kBF16) v_launch<128, kBF16>(a, blocks, s);
   else if (D == 128) v_launch<128, kFP32>(a, blocks, s);
   else if (dtype == kBF16) v_launch<64, kBF16>(a, blocks, s);

@@ -124,3 +124,14 @@ def test_shared_exponent_integer_rule_matches_the_oracle(rule, qmax):
     got = _probe(binding.PROBE_SCALE_EXP, amax, binding.Opts(scale_rule=rule, qmax=qmax))
     ref = np.array([oracle.scale_exponent(float(a), rule, qmax) for a in amax])
     assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("op", [binding.PROBE_E2M1_STANDIN, binding.PROBE_E2M1_MUFU])
+def test_e2m1_code_of_exp2_exact_at_integers(op):
+    """A score equal to the running max gives 2^(0 - e) = 2^-e exactly in the oracle (exp(0) = 1
+    scaled by a power of two); at e = 2 that is the E2M1 midpoint 0.25, which rounds to the even
+    code 0.  Both exponential paths must give the exact code at every integer argument."""
+    u = np.arange(-12, 5, dtype=np.float32)
+    got = _probe(op, u)
+    assert np.array_equal(got, e2m1_code_exact(np.exp2(u.astype(np.float64))))
+    assert got[u == -2][0] == 0 and got[u == -1][0] == 1
