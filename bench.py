@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4"],
                     help="element format: the method's MXFP4, or the NVFP4 comparison format")
-    ap.add_argument("--key-tile", type=int, default=64, choices=[64, 128],
+    ap.add_argument("--key-tile", type=int, default=128, choices=[64, 128],
                     help="keys per online-softmax step (the attention kernel's key tile)")
     ap.add_argument("--causal", action="store_true",
                     help="causal self-attention; TFLOPS count the visible (query, key) pairs, N(N+1)/2 per head")
@@ -77,24 +77,30 @@ def peaks():
         return FALLBACK_BF16_TFLOPS, 6650.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_name(key_tile: int) -> str:
+    return "mxattn_fwd_wide_kernel" if key_tile == 128 else "mxattn_fwd_kernel"
+
+
+def kernel_source_hash(key_tile: int = 128) -> str:
+    """Hash of the sources of the attention kernel for the key tile (and of the shared headers)."""
     h = hashlib.sha256()
-    for name in ("attn.cu", "ptx.cuh", "kernels.cuh"):
+    for name in ("attn_wide.cu" if key_tile == 128 else "attn.cu", "ptx.cuh", "kernels.cuh"):
         with open(os.path.join(ROOT, "mxfp4_bit_attention_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
+def recorded_traffic(workload: str, key_tile: int = 128):
+    """DRAM bytes per attention launch from the committed ncu summary of the kernel for the key
+    tile, if it was taken on that kernel's current source (else None)."""
     path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_source_hash") != kernel_source_hash():
+    rec = rec.get(kernel_name(key_tile), {})
+    if rec.get("kernel_source_hash") != kernel_source_hash(key_tile):
         return None
     per = rec.get("per_workload", {}).get(workload)
     return None if per is None else float(per)
@@ -303,6 +309,8 @@ def main():
     hq, hk, hv = (host_tensor(g[n]) for n in "qkv")
     del g
     q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    if args.format == "nvfp4":
+        args.key_tile = 64  # the NVFP4 comparison format runs with 64-key tiles
     opts = binding.Opts(causal=args.causal, key_tile=args.key_tile,
                         format=binding.FMT_NVFP4 if args.format == "nvfp4" else binding.FMT_MXFP4)
     scale = float(np.float32(w.d ** -0.5))
@@ -385,8 +393,9 @@ def main():
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak,
                 # the recorded DRAM bytes are those of the full-attention MXFP4 kernel
-                "traffic": recorded_traffic(w.name) if (args.format == "mxfp4" and not args.causal) else None,
-                "kernel": "mxattn_fwd_kernel", "ms_per_launch": attn_ms_max,
+                "traffic": recorded_traffic(w.name, args.key_tile) if (args.format == "mxfp4" and not args.causal)
+                else None,
+                "kernel": kernel_name(args.key_tile), "ms_per_launch": attn_ms_max,
                 "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
                 "frac_of_spec_9pf": achieved / 9000.0,
                 "quantizers_ms": quant_ms,

@@ -47,12 +47,29 @@ constexpr int kBN = 128;   // keys per tile
 enum { kModeFull = 0, kModeDump = 1, kModeMasked = 2 };
 constexpr int kStages = 5;  // K/V shared-memory ring depth
 constexpr int kPBufs = 4;   // P^ buffers (tile j uses j % 4)
-constexpr int kProducerWarp = 8, kQkWarp = 9, kPvWarp = 11;  // warps 9 and 10 issue QK for groups 0 and 1
-constexpr int kWarps = 12;
+// Softmax groups: group g (warps 4g..4g+3) takes the key tiles j with j % kGroups == g.  (A third
+// group would need the registers of 128 scores per thread in 16 warps, more than a CTA has.)
+constexpr int kGroups = 2;
+constexpr int kSoftWarps = 4 * kGroups;
+// the warpgroup after the softmax warps: the producer, two QK issuers (tiles of even and odd
+// index, S buffer j % 2) and the PV issuer
+constexpr int kProducerWarp = kSoftWarps, kQkWarp = kSoftWarps + 1, kPvWarp = kSoftWarps + 3;
+constexpr int kWarps = kSoftWarps + 4;
 constexpr int kThreads = 32 * kWarps;
+// S_FULL barriers: tile j commits to j % kSFullSlots, so that a group testing its next tile
+// (kGroups ahead) never sees an older phase of the same barrier
+constexpr int kSFullSlots = 2 * kGroups;
+
 constexpr int kOnesRows = 16;  // rows appended to each 64-key half of V^: row 0 all ones, rows 1..15 zero
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kDrainBudgetCycles = 2000000000LL;
+// Suspend-time hint of the producer's and the MMA issuers' waits (nanoseconds): their work has a
+// tile or more of slack, and a sleeping warp leaves its SM sub-partition's issue slots to the
+// softmax warps there.
+#ifndef MXATTN_ISSUER_SLEEP_NS
+#define MXATTN_ISSUER_SLEEP_NS 1000
+#endif
+constexpr uint32_t kIssuerSleepNs = MXATTN_ISSUER_SLEEP_NS;
 // 8-key words (of the 16 in a tile, word i = keys 8i..8i+7) whose exponentials come from the
 // FMA-pipe stand-in instead of MUFU; PNQ only (direct placement needs the exact exponentials).
 #ifndef MXATTN_WIDE_POLY_MASK
@@ -81,18 +98,18 @@ struct Layout {
   static constexpr int SF_K = SF_ONES + 512;
   static constexpr int SF_V = SF_K + kStages * 512;
   static constexpr int MX = SF_V + kStages * 512;     // running max handed between the groups [128]
-  static constexpr int LX = MX + 512;                 // epilogue, direct placement: l and its frame [2][2][128]
-  static constexpr int BARS = LX + 2048;
+  static constexpr int LX = MX + 512;                 // epilogue: per group l and its frame [kGroups][2][128]
+  static constexpr int BARS = LX + 1024 * kGroups;
   enum {
     B_Q = 0,
     B_KV_FULL = 1,
     B_KV_EMPTY = 1 + kStages,
-    B_S_FULL = 1 + 2 * kStages,  // two: one per S buffer (= softmax group)
-    B_S_FREE = B_S_FULL + 2,     // two
+    B_S_FULL = 1 + 2 * kStages,  // kSFullSlots
+    B_S_FREE = B_S_FULL + kSFullSlots,  // two: one per S buffer (tile parity)
     B_P_FULL = B_S_FREE + 2,     // kPBufs
     B_O_DONE = B_P_FULL + kPBufs,  // kPBufs: PV(j) commits to O_DONE[j % kPBufs]
-    B_XCH = B_O_DONE + kPBufs,   // [2 source groups][4 warp pairs]: running max handed over
-    B_EPI = B_XCH + 8,           // both groups ready for the epilogue
+    B_XCH = B_O_DONE + kPBufs,   // [source group][4 warp quadrants]: running max handed over
+    B_EPI = B_XCH + 4 * kGroups,  // every group ready for the epilogue
     B_DRAIN = B_EPI + 1,
     NUM_BARS
   };
@@ -240,16 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       mbar_init(bar(L::B_KV_FULL + s), 1);
       mbar_init(bar(L::B_KV_EMPTY + s), 1);
     }
-    for (int g = 0; g < 2; g++) {
-      mbar_init(bar(L::B_S_FULL + g), 1);
-      mbar_init(bar(L::B_S_FREE + g), 4);
-    }
+    for (int i = 0; i < kSFullSlots; i++) mbar_init(bar(L::B_S_FULL + i), 1);
+    for (int b = 0; b < 2; b++) mbar_init(bar(L::B_S_FREE + b), 4);
     for (int b = 0; b < kPBufs; b++) {
       mbar_init(bar(L::B_P_FULL + b), 4);
       mbar_init(bar(L::B_O_DONE + b), 1);
     }
-    for (int i = 0; i < 8; i++) mbar_init(bar(L::B_XCH + i), 1);
-    mbar_init(bar(L::B_EPI), 8);
+    for (int i = 0; i < 4 * kGroups; i++) mbar_init(bar(L::B_XCH + i), 1);
+    mbar_init(bar(L::B_EPI), kSoftWarps);
     mbar_init(bar(L::B_DRAIN), 3);  // one commit from each issuer
     fence_mbar_init();
   }
@@ -287,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       for (int j = 0; j < TJ; j++) {
         const int s = j % kStages;
         if (j >= kStages) {
-          ok = mbar_wait(bar(L::B_KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, a.wait_budget);
+          ok = mbar_wait_sleep(bar(L::B_KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, a.wait_budget, kIssuerSleepNs);
           if (!ok) break;
         }
         // the second 64-key half of V^ exists in memory unless the keys end in the first one (its
@@ -319,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     const int g = warp - kQkWarp;
     const bool leader = lane == 0;
     const uint32_t t_sfq = tmem + L::T_SFQ + 4 * g;  // this issuer's own copy of the Q scales
-    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_Q), 0, abort_flag, a.wait_budget));
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_Q), 0, abort_flag, a.wait_budget, kIssuerSleepNs));
     if (ok) {
       tc_fence_after();
       if (leader) tmem_cp_sf_atom(t_sfq, sb + L::SF_Q);
@@ -327,14 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       const uint64_t qdesc = smem_desc(sb + L::Q_CODES, 16, 8 * (D / 2), L::QK_LAYOUT);
       for (int j = g; j < TJ; j += 2) {
         const int s = j % kStages, f = 2 * g + ((j >> 1) & 1);
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
         if (!ok) break;
         tc_fence_after();
         // K scale slot f was last read by QK(j-4), complete since group g read that S before
         // releasing it, which this warp waited for before issuing QK(j-2)
         if (leader) tmem_cp_sf_atom(tmem + L::T_SFK + 4 * f, sb + L::SF_K + 512 * s);
         if (j >= 2) {  // S buffer g was last read by group g at tile j-2
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_S_FREE + g), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_S_FREE + g), ((j - 2) >> 1) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
           if (!ok) break;
           tc_fence_after();
         }
@@ -350,12 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
           // complete before committing S(j).  Each O_DONE barrier is at most one phase away here:
           // PV(j) needs S(j), and this issuer saw PV(j-8) complete before committing S(j-4).
           const int pb = j % kPBufs;
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + pb), ((j - kPBufs) / kPBufs) & 1, abort_flag,
-                                                 a.wait_budget));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_O_DONE + pb), ((j - kPBufs) / kPBufs) & 1, abort_flag,
+                                                       a.wait_budget, kIssuerSleepNs));
           if (!ok) break;
           tc_fence_after();
         }
-        if (leader) mma_commit(bar(L::B_S_FULL + g));
+        if (leader) mma_commit(bar(L::B_S_FULL + j % kSFullSlots));
         __syncwarp();
       }
     }
@@ -375,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       const int s = j % kStages, f = j % L::V_SLOTS, pb = j % kPBufs;
       // V^(j) landed with K^(j), before S(j) and so before P(j); this warp also waits for the stage
       // itself (it cannot have been refilled: that needs this warp's commit below)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
       if (!ok) break;
       tc_fence_after();
       if (leader) {
@@ -386,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         if (PNQ && D == 64) fence_proxy_async_smem();
         tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f, sb + L::SF_V + 512 * s);
       }
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_P_FULL + pb), (j / kPBufs) & 1, abort_flag, a.wait_budget));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_P_FULL + pb), (j / kPBufs) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
       if (!ok) break;
       tc_fence_after();
       if (leader) {
@@ -411,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     if (leader) mma_commit(bar(L::B_DRAIN));
     __syncwarp();
     mbar_wait(bar(L::B_DRAIN), 0, no_abort, kDrainBudgetCycles);
-  } else if (warp < 8) {
+  } else if (warp < kSoftWarps) {
     // ------------------------------------------------------------------ softmax (warps 0-7)
-    const int grp = warp >> 2;             // softmax group: key tiles j with j % 2 == grp
+    const int grp = warp >> 2;             // softmax group: key tiles j with j % kGroups == grp
     const int quad = warp & 3;             // TMEM lane quadrant = the warp pair's 32 query rows
     const int row = quad * 32 + lane;      // TMEM lane and query row within the tile
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
@@ -428,20 +443,22 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     bool ok = true;
     bool s_ready = false;   // S(j) was seen complete by the early test during tile j-2
     // one key tile; FULL: all 128 keys are inside this row's range, so the body carries no masking
-    auto tile = [&](int j, auto full_tag) -> bool {
+    const float tau = a.tau, log2q = a.rule.log2q;
+    auto tile = [&](int j, auto full_tag, auto floor_tag) -> bool {
       constexpr bool FULL = decltype(full_tag)::value;
+      constexpr bool FLOOR = decltype(floor_tag)::value;  // the OCP floor scale rule
       if (!__all_sync(0xFFFFFFFFu, s_ready)) {
-        ok = mbar_wait(bar(L::B_S_FULL + grp), (j >> 1) & 1, abort_flag, a.wait_budget);
+        ok = mbar_wait(bar(L::B_S_FULL + j % kSFullSlots), (j / kSFullSlots) & 1, abort_flag, a.wait_budget);
         if (!__all_sync(0xFFFFFFFFu, ok)) return false;
       }
       tc_fence_after();
-      const uint32_t sbuf = tl + L::T_S + 128 * grp;
+      const uint32_t sbuf = tl + L::T_S + 128 * (j & 1);
       uint32_t s[128];
       tmem_ld128_wait(sbuf, s);
       // S(j) is in registers: the QK MMA of tile j+2 may overwrite the buffer
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_S_FREE + grp));
+      if (lane == 0) mbar_arrive(bar(L::B_S_FREE + (j & 1)));
       if (!FULL) {
         const int valid = kmax - j * kBN;  // this row's keys in the tile (may be <= 0)
 #pragma unroll
@@ -455,23 +472,45 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       float gmax[4];
       group_maxima(s, gmax);
       const float mt_raw = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3]));
-      // the running max after tile j-1, handed over by the other group
+      // Lazy running max (threshold tau, log2 units): the max moves only when the tile's max
+      // exceeds the running max before the tile by more than tau.
+      // The codes depend on the running max after this tile (their frame).  A group's maximum is
+      // taken as 2^((gmax - frame) * c): exactly 1 for the group that holds the running max, as
+      // exp(0) is in the oracle.
+      uint32_t eb[4], w[16];
+      float psum[4];
+      auto codes = [&](float fr) {
+        float ex[4];  // the groups' shared exponents e
+#pragma unroll
+        for (int g = 0; g < 4; g++) {
+          ex[g] = shared_exponent_log2f_rule<FLOOR>((gmax[g] - fr) * c, log2q, eb[g]);
+          psum[g] = 0.f;
+        }
+        group_codes<0, PNQ>(s, fr, c, ex[0], w, psum[0]);
+        group_codes<1, PNQ>(s, fr, c, ex[1], w + 4, psum[1]);
+        group_codes<2, PNQ>(s, fr, c, ex[2], w + 8, psum[2]);
+        group_codes<3, PNQ>(s, fr, c, ex[3], w + 12, psum[3]);
+      };
+      // The running max before this tile is the one after tile j-1, which the other group hands
+      // over.  Rather than wait for it, take this group's own last running max (the one after tile
+      // j-2, unchanged unless the other group moved it) and code the tile in that frame; then check
+      // the frame against the handed-over max and code again only where it differs (moves are
+      // rare under the lazy rule), so the hand-over stays off the critical path.
       float sm_prev = -INFINITY;
       if (j > 0) {
-        ok = mbar_wait(bar(L::B_XCH + 4 * (grp ^ 1) + quad), ((j - 1) >> 1) & 1, abort_flag, a.wait_budget);
+        ok = mbar_wait(bar(L::B_XCH + 4 * ((grp + kGroups - 1) % kGroups) + quad), ((j - 1) / kGroups) & 1,
+                       abort_flag, a.wait_budget);
         if (!__all_sync(0xFFFFFFFFu, ok)) return false;
         sm_prev = mx[row];
       }
-      // Lazy running max (threshold tau, log2 units): the max moves only when the tile's max
-      // exceeds it by more than tau.  A group's maximum is taken as 2^((gmax - sm) * c): exactly 1
-      // for the group that holds the running max, as exp(0) is in the oracle.
-      const bool move = j == 0 || (mt_raw * c > sm_prev * c + a.tau);
+      const bool move = j == 0 || (mt_raw * c > sm_prev * c + tau);
       const float sm_new = move ? mt_raw : sm_prev;
       if (j + 1 < TJ) {  // hand the max on as early as possible: the other group waits for it
         mx[row] = sm_new;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_XCH + 4 * grp + quad));
       }
+      codes(sm_new);
       const float m2 = sm_new * c;
       // O~ and l are rescaled by alpha = 2^(m_old - m_new) only when some row of the warp moves
       // its max (alpha = 1 elsewhere); tile 0 starts both at zero
@@ -480,23 +519,13 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       if (any_move && move) alpha = ex2_approx((sm_prev - sm_new) * c);
       if (!PNQ && sm != sm_new) l *= ex2_approx((sm - sm_new) * c);  // this group's l into the new frame
       sm = sm_new;
-
-      uint32_t eb[4];
-      float ex[4];  // the groups' shared exponents e
-#pragma unroll
-      for (int g = 0; g < 4; g++) ex[g] = shared_exponent_log2f((gmax[g] - sm_new) * c, a.rule, eb[g]);
-      uint32_t w[16];
-      float psum[4] = {0.f, 0.f, 0.f, 0.f};
-      group_codes<0, PNQ>(s, sm_new, c, ex[0], w, psum[0]);
-      group_codes<1, PNQ>(s, sm_new, c, ex[1], w + 4, psum[1]);
-      group_codes<2, PNQ>(s, sm_new, c, ex[2], w + 8, psum[2]);
-      group_codes<3, PNQ>(s, sm_new, c, ex[3], w + 12, psum[3]);
       if (dumping) {  // the unquantized tile, relative to this tile's running max
         float* dpt = reinterpret_cast<float*>(a.dump + dl.p_tilde) + ((size_t)j * 128 + row) * kBN;
         for (int i = 0; i < 128; i++) dpt[i] = ex2_approx((__uint_as_float(s[i]) - sm_new) * c);
       }
       // test S(j+2) now, so that the test's latency overlaps the stores below
-      s_ready = j + 2 < TJ && mbar_test(bar(L::B_S_FULL + grp), ((j + 2) >> 1) & 1);
+      s_ready = j + kGroups < TJ &&
+                mbar_test(bar(L::B_S_FULL + (j + kGroups) % kSFullSlots), ((j + kGroups) / kSFullSlots) & 1);
       if (!PNQ) {
 #pragma unroll
         for (int g = 0; g < 4; g++) l += psum[g] * __uint_as_float(eb[g] << 23);  // byte 0: 2^-127 -> 0
@@ -555,13 +584,17 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     // keys; under causal masking the diagonal tile)
     int full_tiles = (Nk % kBN == 0) ? T : T - 1;
     if (causal && full_tiles > qt) full_tiles = qt;
-    int j = grp;
-    for (; ok && j < full_tiles; j += 2) ok = tile(j, std::true_type{});
-    for (; ok && j < TJ; j += 2) ok = tile(j, std::false_type{});
+    auto sweep = [&](auto floor_tag) {
+      int j = grp;
+      for (; ok && j < full_tiles; j += kGroups) ok = tile(j, std::true_type{}, floor_tag);
+      for (; ok && j < TJ; j += kGroups) ok = tile(j, std::false_type{}, floor_tag);
+    };
+    if (a.rule.mq == 0xFFFFFFFFu) sweep(std::true_type{});
+    else sweep(std::false_type{});
 
     // Epilogue.  The group that ran the last tile knows PV(TJ-5) complete (S(TJ-1) was committed
     // after it), so its wait on PV(TJ-1)'s barrier is unambiguous; it then lets the other group in.
-    const int last_grp = (TJ - 1) & 1;
+    const int last_grp = (TJ - 1) % kGroups;
     if (ok && grp == last_grp) {
       const int pb = (TJ - 1) % kPBufs;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(L::B_O_DONE + pb), ((TJ - 1) / kPBufs) & 1, abort_flag, a.wait_budget));
@@ -590,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         lsum = __uint_as_float(lv);
       } else {
         lsum = 0.f;
-        for (int g = 0; g < 2; g++) {
+        for (int g = 0; g < kGroups; g++) {
           const float lg = lx[g * 256 + row];
           if (lg != 0.f) lsum += lg * ex2_approx((lx[g * 256 + 128 + row] - sm_final) * c);
         }
@@ -603,9 +636,9 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         reinterpret_cast<float*>(a.dump + dl.l)[row] = lsum;
         reinterpret_cast<float*>(a.dump + dl.m)[row] = sm_final * c;
       }
-      // each group writes half of the row's D outputs
+      // the groups share the row's D outputs, 32 columns at a time
 #pragma unroll 1
-      for (int cc = grp * (D / 64); cc < (grp + 1) * (D / 64); cc++) {
+      for (int cc = grp; cc < D / 32; cc += kGroups) {
         uint32_t o[32];
         tmem_ld32(tl + L::T_O + 32 * cc, o);
         tmem_wait_ld();

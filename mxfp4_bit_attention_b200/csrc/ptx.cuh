@@ -109,6 +109,34 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint (nanoseconds): the thread sleeps until the phase completes
+// or the hint expires, issuing nothing meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for warps whose work has slack (the producer and the MMA issuers): each try
+// may sleep up to `hint_ns`, so a waiting warp takes almost no issue slots from the warps that
+// share its SM sub-partition.  Gives up as mbar_wait does.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                                long long budget, uint32_t hint_ns) {
+  if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > budget) return false;
+  }
+}
+
 // Bounded wait.  Gives up (returns false) after `budget` SM clock cycles, or as
 // soon as *abort becomes non-zero (another warp gave up first).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
@@ -333,6 +361,38 @@ __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[12
       : "memory");
 }
 
+// The same load without the wait: the registers hold the columns only after tmem_wait_ld(), and
+// every use must be pinned below that wait (pin1 on each register).
+__device__ __forceinline__ void tmem_ld128_nowait(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
+      "%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,"
+      "%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,"
+      "%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,"
+      "%126,%127}, [%128];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+        "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]),
+        "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]),
+        "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]),
+        "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void pin32(uint32_t (&r)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; i++) pin1(r[i]);
@@ -489,16 +549,22 @@ struct ScaleRule {
 // (ceiling rules) or -inf (floor rule) lands on the integer M + ceil(x) or M + floor(x), in a
 // binade whose ulp is 1, so the sum's low mantissa bits are 127 + e.  Clamping x to
 // [-127, 127] first (an integer range) clamps e the same way; t = -inf gives -127.
-__device__ __forceinline__ float shared_exponent_log2f(float t, ScaleRule r, uint32_t& byte) {
+template <bool FLOOR>  // FLOOR: the OCP floor rule; else a ceiling rule with boundary 2^log2q
+__device__ __forceinline__ float shared_exponent_log2f_rule(float t, float log2q, uint32_t& byte) {
   constexpr float M = 12582912.f + 127.f;
   float y;
-  if (r.mq == 0xFFFFFFFFu) {  // floor(t) - 2: floor t itself (t - 2 could round), M - 2 adds the -2
+  if (FLOOR) {  // floor(t) - 2: floor t itself (t - 2 could round), M - 2 adds the -2
     y = __fadd_rd(fminf(fmaxf(t, -125.f), 129.f), M - 2.f);
   } else {
-    y = __fadd_ru(fminf(fmaxf(t - r.log2q, -127.f), 127.f), M);
+    y = __fadd_ru(fminf(fmaxf(t - log2q, -127.f), 127.f), M);
   }
   byte = __float_as_uint(y) & 0xFFu;
   return y - M;
+}
+
+__device__ __forceinline__ float shared_exponent_log2f(float t, ScaleRule r, uint32_t& byte) {
+  return r.mq == 0xFFFFFFFFu ? shared_exponent_log2f_rule<true>(t, r.log2q, byte)
+                             : shared_exponent_log2f_rule<false>(t, r.log2q, byte);
 }
 
 __device__ __forceinline__ int shared_exponent(float amax, ScaleRule r) {

@@ -48,15 +48,17 @@ def test_recorded_traffic_is_keyed_to_the_kernel_source(tmp_path, monkeypatch):
     """The committed DRAM-traffic record is used only while the kernel sources hash to the value it
     was captured on; any other source gives no traffic figure."""
     b = _bench_module()
-    rec = {"kernel_source_hash": "0123456789abcdef", "per_workload": {"720p": 1.25e9, "480p": 5.5e8}}
+    rec = {"mxattn_fwd_wide_kernel": {"kernel_source_hash": "0123456789abcdef",
+                                      "per_workload": {"720p": 1.25e9, "480p": 5.5e8}}}
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "attn_fwd_traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(b, "ROOT", str(tmp_path))
-    monkeypatch.setattr(b, "kernel_source_hash", lambda: "0123456789abcdef")
-    assert b.recorded_traffic("720p") == 1.25e9
-    assert b.recorded_traffic("joint") is None
-    monkeypatch.setattr(b, "kernel_source_hash", lambda: "ffffffffffffffff")
-    assert b.recorded_traffic("720p") is None
+    monkeypatch.setattr(b, "kernel_source_hash", lambda key_tile=128: "0123456789abcdef")
+    assert b.recorded_traffic("720p", 128) == 1.25e9
+    assert b.recorded_traffic("joint", 128) is None
+    assert b.recorded_traffic("720p", 64) is None  # no record for the 64-key kernel
+    monkeypatch.setattr(b, "kernel_source_hash", lambda key_tile=128: "ffffffffffffffff")
+    assert b.recorded_traffic("720p", 128) is None
 
 
 def test_gpus_n_without_torchrun_starts_n_ranks():
