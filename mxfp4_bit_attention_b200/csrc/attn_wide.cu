@@ -492,10 +492,9 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         group_codes<3, PNQ>(s, fr, c, ex[3], w + 12, psum[3]);
       };
       // The running max before this tile is the one after tile j-1, which the other group hands
-      // over.  Rather than wait for it, take this group's own last running max (the one after tile
-      // j-2, unchanged unless the other group moved it) and code the tile in that frame; then check
-      // the frame against the handed-over max and code again only where it differs (moves are
-      // rare under the lazy rule), so the hand-over stays off the critical path.
+      // over through shared memory (its XCH barrier); the codes are formed in the frame after this
+      // tile, so they wait for it.  The hand-over is published right after the maxima, before
+      // this group's own codes, so the other group's wait is short.
       float sm_prev = -INFINITY;
       if (j > 0) {
         ok = mbar_wait(bar(L::B_XCH + 4 * ((grp + kGroups - 1) % kGroups) + quad), ((j - 1) / kGroups) & 1,

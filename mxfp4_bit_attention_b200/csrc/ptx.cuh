@@ -261,6 +261,19 @@ __device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t smem_at
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (cp.async, L2 only): src_bytes 16 copies, 0 fills
+// the 16 bytes with zeros (src is not read).  Both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// every cp.async of this thread has landed (visible to the thread; a barrier publishes them)
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// close the thread's current group of cp.async copies
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most N of the thread's committed groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Warp-collective TMEM loads / stores: lane i of warp w (w = warp index mod 4) touches TMEM lane
 // 32*w + i; 32 consecutive 32-bit columns starting at taddr's column.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

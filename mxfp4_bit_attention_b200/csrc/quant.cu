@@ -1,6 +1,7 @@
 // quant.cu -- MXFP4 quantizers (rotation + quantization of Q/K, V along keys, and a plain
 // generic quantizer).  Memory-bound: every byte is read once and written once, loads and
-// stores are 16-byte vectors, FWHT butterflies run in registers and warp shuffles.
+// stores are 16-byte vectors (inputs staged through shared memory by cp.async), and the FWHT
+// butterflies of a row run in one thread's registers.
 //
 // Method: "MXAttention: Data-Free Optimal Scaling and Pre-Normalization Quantization for
 // MXFP4 Attention" -- Pith review page (axioms ledger: 32-element E2M1 groups with one E8M0
@@ -16,29 +17,6 @@
 #include "ptx.cuh"
 
 namespace mxattn {
-
-template <int DT>
-__device__ __forceinline__ void load8(const void* base, int64_t idx, bool valid, float (&v)[8]) {
-  if (!valid) {
-#pragma unroll
-    for (int i = 0; i < 8; i++) v[i] = 0.f;
-    return;
-  }
-  if (DT == kBF16) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-      v[2 * i] = __uint_as_float(w[i] << 16);
-      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
-    const float4 a = p[0], b = p[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
-}
 
 // One NVFP4 block of 16 values (the comparison format): the scale is the E4M3 rounding of
 // fl32(amax / 6), each value is divided by it in fp32 (correctly rounded) and rounded to E2M1
@@ -59,99 +37,63 @@ __device__ __forceinline__ uint32_t nvfp4_block(const float* v, uint32_t* w) {
 
 // ------------------------------------------------------------------------------------------------
 // Q/K: Hadamard rotation + quantization along d into the packed QK operand layout.
-// One thread per MX group (32 consecutive elements of a row, four 16-byte loads in flight), D/32
-// threads per row: butterfly stages h = 1..16 run inside the thread, h = 32 and 64 across the
-// row's threads by shuffles, in the order h = 1, 2, ..., D/2; the group max is the thread's own.
-// Grid: x over (B*H*T128*128) padded token rows of the longer of Q and K, y = 0 for Q, 1 for K;
-// varlen: over H * tiles_per_head * 128 padded rows, each tile belonging to one sequence.
+// One thread per padded token row: the row's D values are staged through shared memory (16-byte
+// cp.async copies of the block's rows, zeros for padding rows), then the thread runs every
+// butterfly stage h = 1, 2, ..., D/2 of the fast Walsh-Hadamard transform in registers, scales by
+// fl32(1/sqrt(D)), and quantizes its D/32 groups.  No value crosses threads, so the row needs no
+// shuffles.  Grid: x over the 128-row packed tiles of the longer of Q and K (SPLIT blocks per
+// tile), y = 0 for Q, 1 for K; varlen: over H * tiles_per_head tiles, each tile belonging to one
+// sequence.
 // ------------------------------------------------------------------------------------------------
-// Where padded row prow of the Q or K operand comes from: its row of the [rows, D] source (valid: a
-// real token; a padding row is quantized from zeros) and its packed tile and row within the tile.
-struct QKRow {
-  bool ok, valid;
-  int64_t src_row, tile;
-  int r;
+// Where the rows of packed tile `tile` (bh * T128 + tile within the head) come from: rows r <
+// nvalid are source rows src_row0 + r * stride of the [rows, D] input; the rest are padding.
+struct QKTile {
+  bool ok;  // the tile exists (varlen: tiles past the last sequence's are unused)
+  int nvalid;
+  int64_t src_row0, stride;
 };
 
-__device__ __forceinline__ QKRow qk_row(const QKQuantArgs& a, int64_t prow, int64_t total, int64_t T128, int Nt) {
-  QKRow q;
-  q.ok = prow < total;
-  const int64_t bh = prow / (T128 * 128);
-  q.r = (int)(prow % 128);
-  q.tile = prow / 128;  // bh * T128 + tile within the head
+__device__ __forceinline__ QKTile qk_tile(const QKQuantArgs& a, uint32_t tile, uint32_t T128, int Nt) {
+  QKTile q;
+  const uint32_t bh = tile / T128;  // tile counts fit 32 bits (the grid is one-dimensional)
+  const int tt = (int)(tile - bh * T128);
+  q.ok = bh < (uint32_t)a.BH;
   if (a.vl.cu_seqlens != nullptr) {
-    // the tile's sequence and the row's token within it; tiles past the last sequence's are unused
-    const int gt = (int)(q.tile - bh * T128);
-    q.ok = q.ok && gt < __ldg(a.vl.tile_off + a.vl.nseq);
-    const int sq = q.ok ? varlen_sequence(a.vl, gt) : 0;
+    q.ok = q.ok && tt < __ldg(a.vl.tile_off + a.vl.nseq);
+    const int sq = q.ok ? varlen_sequence(a.vl, tt) : 0;
     const int start = __ldg(a.vl.cu_seqlens + sq);
-    const int n = (gt - __ldg(a.vl.tile_off + sq)) * 128 + q.r;
-    q.valid = q.ok && n < __ldg(a.vl.cu_seqlens + sq + 1) - start;
-    q.src_row = ((int64_t)start + n) * a.BH + bh;  // token-major [T, H, d]
+    const int n0 = (tt - __ldg(a.vl.tile_off + sq)) * 128;
+    const int len = __ldg(a.vl.cu_seqlens + sq + 1) - start;
+    q.nvalid = len - n0 < 0 ? 0 : (len - n0 > 128 ? 128 : len - n0);
+    q.src_row0 = ((int64_t)start + n0) * a.BH + (int64_t)bh;  // token-major [T, H, d]
+    q.stride = a.BH;
   } else {
-    const int tok = (int)(prow % (T128 * 128));
-    q.valid = q.ok && tok < Nt;
-    q.src_row = (int64_t)bh * Nt + tok;
+    const int tok0 = tt * 128;
+    q.nvalid = Nt - tok0 < 0 ? 0 : (Nt - tok0 > 128 ? 128 : Nt - tok0);
+    q.src_row0 = (int64_t)bh * Nt + tok0;
+    q.stride = 1;
   }
   return q;
 }
 
-// The 32 inputs of one thread's group as loaded (bf16: four 16-byte words; fp32: eight).
-template <int DT>
-struct GroupRaw {
-  uint4 w[DT == kBF16 ? 4 : 8];
-};
-
-template <int DT>
-__device__ __forceinline__ void load_group(const void* src, int64_t idx, bool valid, GroupRaw<DT>& raw) {
-  constexpr int NW = DT == kBF16 ? 4 : 8;
-  const uint4* p = DT == kBF16 ? reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + idx)
-                               : reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(src) + idx);
+// In-place fast Walsh-Hadamard transform of one row, stages h = 1, ..., D/2, each butterfly
+// (x, y) -> (x + y, x - y) rounded once (x - y as fma(y, -1, x)); from h = 2 on, neighbours i,
+// i+1 pair up into f32x2 operations with the same roundings.  The multiply by fl32(1/sqrt(D))
+// that ends the rotation is left to the quantizer (rotate_quant_qk_kernel), which folds it into
+// the group's scaling where that is exact.
+template <int D>
+__device__ __forceinline__ void fwht_row(float (&v)[D]) {
 #pragma unroll
-  for (int i = 0; i < NW; i++) raw.w[i] = valid ? p[i] : make_uint4(0u, 0u, 0u, 0u);
-}
-
-template <int DT>
-__device__ __forceinline__ void unpack_group(const GroupRaw<DT>& raw, float (&v)[32]) {
-  if (DT == kBF16) {
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const uint32_t w[4] = {raw.w[i].x, raw.w[i].y, raw.w[i].z, raw.w[i].w};
-#pragma unroll
-      for (int k = 0; k < 4; k++) {
-        v[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-        v[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      v[4 * i] = __uint_as_float(raw.w[i].x);
-      v[4 * i + 1] = __uint_as_float(raw.w[i].y);
-      v[4 * i + 2] = __uint_as_float(raw.w[i].z);
-      v[4 * i + 3] = __uint_as_float(raw.w[i].w);
-    }
-  }
-}
-
-// Hadamard rotation of one row held by its TPR = D/32 lanes, 32 values each, in place: butterfly
-// stages h = 1..16 inside the thread, h = 32..D/2 across the row's lanes by shuffles, then the
-// multiply by fl32(1/sqrt(D)).  Every lane of the warp must take part (the shuffles are full-warp).
-template <int TPR>
-__device__ __forceinline__ void rotate_group(float (&v)[32], int g, float hadamard_scale) {
-  // Butterflies (x, y) -> (x + y, x - y), each result rounded once: x - y as fma(y, -1, x).
-  // From h = 2 on, neighbours i, i+1 pair up into f32x2 operations with the same roundings.
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
+  for (int i = 0; i < D; i += 2) {
     const float x = v[i], y = v[i + 1];
     v[i] = __fadd_rn(x, y);
     v[i + 1] = __fsub_rn(x, y);
   }
   const float2 minus1 = make_float2(-1.f, -1.f);
 #pragma unroll
-  for (int h = 2; h < 32; h <<= 1) {
+  for (int h = 2; h < D; h <<= 1) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
+    for (int i = 0; i < D; i += 2) {
       if ((i & h) == 0) {
         const float2 x = make_float2(v[i], v[i + 1]), y = make_float2(v[i + h], v[i + h + 1]);
         const float2 sum = __fadd2_rn(x, y), dif = __ffma2_rn(y, minus1, x);
@@ -160,99 +102,141 @@ __device__ __forceinline__ void rotate_group(float (&v)[32], int g, float hadama
       }
     }
   }
-  // stages h = 32 .. D/2 across the TPR lanes of the row (lane bit = h / 32): the lower lane
-  // keeps x + y, the upper one y' = x - y, both as fma(own, +-1, other)
+}
+
+// Rows (threads) per block, and the blocks each SM must hold at D = 128 (the register cap that
+// follows, 168 a thread, holds the row's 128 values without spilling).  Measured on the 720p
+// shapes: 64-row blocks six to an SM beat 128-row blocks three to an SM by 5%, and either is
+// a third faster than two 128-row blocks at the registers the compiler would otherwise take.
+constexpr int kQKRows = 64;
+constexpr int kQKBlocksPerSM128 = 6;
+template <int D, int DT>
+struct QKBlock {
+  static constexpr int ES = DT == kBF16 ? 2 : 4;       // bytes per element
+  static constexpr int ROWS = kQKRows;                 // rows per block (threads)
+  static constexpr int SPLIT = 128 / ROWS;             // blocks per packed tile
+  static constexpr int ROWB = D * ES;                  // source bytes per row
+  static constexpr int PITCH = ROWB + 16;              // staged row pitch: rows 4 banks apart
+};
+
+// MXFP4 codes of one group of 32 rotated values x = fl(y * hs) (rotate) or x = y: with
+// e = shared_exponent(max |x|), each code is E2M1(x * 2^-e).  max |x| = fl(max |y| * hs) as
+// rounding is monotone, and fl(y * hs) * 2^-e = fl(y * (hs * 2^-e)) exactly whenever hs * 2^-e is
+// a normal number and y * hs does not underflow; a y * hs that does underflow gives code 0 either
+// way unless e is near -127, and those groups (max |x| below ~2^-97) take the two roundings as
+// the definition states.
+__device__ __forceinline__ int mx_group_codes(float* y, bool rotate, float hs, ScaleRule rule, uint32_t (&w)[4]) {
+  float amax = 0.f;
 #pragma unroll
-  for (int hb = 1; hb < TPR; hb <<= 1) {
-    const float sg = (g & hb) != 0 ? -1.f : 1.f;
-    const float2 sg2 = make_float2(sg, sg);
+  for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(y[i]));
+  if (rotate) amax = __fmul_rn(amax, hs);
+  const int e = shared_exponent(amax, rule);
+  float mul = pow2_neg(e);
+  if (rotate) {
+    if (e > -100) {
+      mul = __fmul_rn(hs, mul);  // exact
+    } else {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const float o0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], hb);
-      const float o1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], hb);
-      const float2 r = __ffma2_rn(make_float2(v[i], v[i + 1]), sg2, make_float2(o0, o1));
-      v[i] = r.x; v[i + 1] = r.y;
+      for (int i = 0; i < 32; i++) y[i] = __fmul_rn(y[i], hs);
     }
   }
-  const float2 hs = make_float2(hadamard_scale, hadamard_scale);
+  const float2 m2 = make_float2(mul, mul);
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), hs);
-    v[i] = r.x; v[i + 1] = r.y;
+  for (int q = 0; q < 4; q++) {
+    float2 p[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) p[k] = __fmul2_rn(make_float2(y[8 * q + 2 * k], y[8 * q + 2 * k + 1]), m2);
+    w[q] = cvt_e2m1x8(p[0].x, p[0].y, p[1].x, p[1].y, p[2].x, p[2].y, p[3].x, p[3].y);
   }
+  return e;
 }
 
 template <int D, int DT, bool NVF>
-__global__ void __launch_bounds__(256) rotate_quant_qk_kernel(QKQuantArgs a) {
-  constexpr int TPR = D / 32;                // threads per row = groups per row
-  constexpr int ROWS = 256 / TPR;            // rows per block and pass
+__global__ void __launch_bounds__(QKBlock<D, DT>::ROWS, kQKBlocksPerSM128) rotate_quant_qk_kernel(QKQuantArgs a) {
+  using B = QKBlock<D, DT>;
+  __shared__ __align__(16) uint8_t stage[B::ROWS * B::PITCH];
   const int t = threadIdx.x;
-  const int g = t % TPR;                     // group (and 16-byte code chunk) within the row
   const int Nt = blockIdx.y == 0 ? a.N : a.Nk;  // tokens of this tensor
-  const int64_t T128 = a.vl.cu_seqlens != nullptr ? a.vl.tiles_per_head : (Nt + 127) / 128;
-  const int64_t total = (int64_t)a.BH * T128 * 128;
-  const void* src = blockIdx.y == 0 ? a.q : a.k;
-  uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
-  uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
-
-  // Grid-stride over passes of ROWS rows (the pass count is the block's, so a row's lanes, which
-  // exchange values by shuffles, always run together); the next pass's inputs are loaded before
-  // this pass's rotation and quantization, so a load is in flight while the thread computes.
-  const int64_t stride = (int64_t)gridDim.x * ROWS;
-  int64_t prow = (int64_t)blockIdx.x * ROWS + t / TPR;
-  QKRow row = qk_row(a, prow, total, T128, Nt);
-  GroupRaw<DT> raw;
-  load_group<DT>(src, (row.valid ? row.src_row : 0) * D + g * 32, row.valid, raw);
-  for (int64_t pass = (int64_t)blockIdx.x * ROWS; pass < total; pass += stride, prow += stride) {
-    const QKRow cur = row;
-    float v[32];
-    unpack_group<DT>(raw, v);
-    if (pass + stride < total) {
-      row = qk_row(a, prow + stride, total, T128, Nt);
-      load_group<DT>(src, (row.valid ? row.src_row : 0) * D + g * 32, row.valid, raw);
-    }
-    if (a.rotate) rotate_group<TPR>(v, g, a.hadamard_scale);
-    uint32_t w[4];
-    int e = 0;
-    uint32_t nvb = 0;  // NVFP4: the two E4M3 scale bytes of the thread's blocks of 16
-    if (NVF) {
-      nvb = nvfp4_block(v, w) | (nvfp4_block(v + 16, w + 2) << 8);
-    } else {
-      float amax = 0.f;
+  const uint32_t T128 = a.vl.cu_seqlens != nullptr ? (uint32_t)a.vl.tiles_per_head : (uint32_t)(Nt + 127) / 128;
+  const uint32_t tile = blockIdx.x / B::SPLIT;
+  const int row0 = (int)(blockIdx.x % B::SPLIT) * B::ROWS;  // first row of the tile this block takes
+  const QKTile qt = qk_tile(a, tile, T128, Nt);
+  if (!qt.ok) return;  // the whole block
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(blockIdx.y == 0 ? a.q : a.k);
+  // stage: consecutive threads copy consecutive 16-byte chunks of a row (coalesced)
 #pragma unroll
-      for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
-      e = shared_exponent(amax, a.rule);
-      const float inv = pow2_neg(e);
+  for (int idx = t; idx < B::ROWS * (B::ROWB / 16); idx += B::ROWS) {
+    const int rr = idx / (B::ROWB / 16), chunk = idx % (B::ROWB / 16);
+    const int r = row0 + rr;
+    const bool valid = r < qt.nvalid;
+    const uint8_t* g = src + (qt.src_row0 + (int64_t)(valid ? r : 0) * qt.stride) * B::ROWB + chunk * 16;
+    cp_async16(smem_u32(stage + rr * B::PITCH + chunk * 16), g, valid ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  float v[D];
+  const uint8_t* mine = stage + t * B::PITCH;
 #pragma unroll
-      for (int q = 0; q < 4; q++)
-        w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
-                          __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
-                          __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
-    }
-    if (!cur.ok) continue;
-    const int r = cur.r;
-    const int sw = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
-    uint8_t* rowp = codes + (cur.tile * 128 + r) * (D / 2);
-    *reinterpret_cast<uint4*>(rowp + ((g ^ sw) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (NVF) {
-      // D/64 scale atoms per tile, one per 64 dims (one K = 64 MMA): blocks 4a..4a+3 in the bytes
-      // of row r's word; this thread's blocks 2g, 2g+1 sit in atom g/2, bytes 2(g%2), 2(g%2)+1
-      uint8_t* atom = scales + cur.tile * (512 * (D / 64)) + (g / 2) * 512 + (r % 32) * 16 + (r / 32) * 4;
-      *reinterpret_cast<uint16_t*>(atom + 2 * (g % 2)) = (uint16_t)nvb;
+  for (int c = 0; c < B::ROWB / 16; c++) {
+    const uint4 w = *reinterpret_cast<const uint4*>(mine + 16 * c);
+    if (DT == kBF16) {
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        v[8 * c + 2 * k] = __uint_as_float(ww[k] << 16);
+        v[8 * c + 2 * k + 1] = __uint_as_float(ww[k] & 0xFFFF0000u);
+      }
     } else {
-      uint8_t* atom = scales + cur.tile * 512 + (r % 32) * 16 + (r / 32) * 4;
-      atom[g] = (uint8_t)(e + 127);
-      if (D == 64) atom[g + 2] = 0;                         // unused scale slots
+      v[4 * c] = __uint_as_float(w.x);
+      v[4 * c + 1] = __uint_as_float(w.y);
+      v[4 * c + 2] = __uint_as_float(w.z);
+      v[4 * c + 3] = __uint_as_float(w.w);
     }
   }
+  const bool rotate = a.rotate != 0;
+  if (rotate) fwht_row<D>(v);
+  const int r = row0 + t;  // row within the tile
+  uint8_t* codes = blockIdx.y == 0 ? a.q_codes : a.k_codes;
+  uint8_t* scales = blockIdx.y == 0 ? a.q_scales : a.k_scales;
+  uint8_t* rowp = codes + ((int64_t)tile * 128 + r) * (D / 2);
+  const int sw = (D == 128) ? ((r >> 1) & 3) : ((r >> 2) & 1);
+  uint32_t sbytes = 0;  // MXFP4: the row's D/32 scale bytes; NVFP4: four block bytes per atom
+#pragma unroll
+  for (int g = 0; g < D / 32; g++) {
+    float* x = v + 32 * g;
+    uint32_t w[4];
+    if (NVF) {
+      if (rotate) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 r2 = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(a.hadamard_scale, a.hadamard_scale));
+          x[i] = r2.x; x[i + 1] = r2.y;
+        }
+      }
+      const uint32_t b = nvfp4_block(x, w) | (nvfp4_block(x + 16, w + 2) << 8);
+      sbytes |= b << (16 * (g % 2));
+      if (g % 2 == 1) {
+        // D/64 scale atoms per tile, one per 64 dims (one K = 64 MMA): blocks 4a..4a+3 in the
+        // bytes of row r's word
+        uint8_t* atom = scales + (int64_t)tile * (512 * (D / 64)) + (g / 2) * 512 + (r % 32) * 16 + (r / 32) * 4;
+        *reinterpret_cast<uint32_t*>(atom) = sbytes;
+        sbytes = 0;
+      }
+    } else {
+      const int e = mx_group_codes(x, rotate, a.hadamard_scale, a.rule, w);
+      sbytes |= (uint32_t)(e + 127) << (8 * g);  // D = 64: bytes 2, 3 (unused slots) stay 0
+    }
+    *reinterpret_cast<uint4*>(rowp + ((g ^ sw) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (!NVF) *reinterpret_cast<uint32_t*>(scales + (int64_t)tile * 512 + (r % 32) * 16 + (r / 32) * 4) = sbytes;
 }
 
 // ------------------------------------------------------------------------------------------------
 // V: quantization along keys (32 consecutive tokens per channel) into the packed V operand
-// layout.  Blocks stride over the (head, 64-key tile) items; each tile is staged through shared
-// memory as fp32 [64][D+1], then thread (channel c, half h) quantizes keys 32h..32h+31 of channel
-// c.  The next tile's inputs are loaded into registers before the current tile is quantized, so
-// a load is always in flight while the block computes.
+// layout.  One block of D threads per (head, 64-key tile): the tile's 64 key rows are copied into
+// shared memory as they are (bf16 or fp32, 16-byte cp.async copies, zeros for keys past the
+// sequence), then thread t quantizes channels 2p, 2p+1 (p = t mod D/2) over keys 32h..32h+31
+// (h = t / (D/2)), reading both channels of a key in one 32- or 64-bit word.
 // Varlen: items over (head, 64-key tile of the packed tiles); each sequence's groups start at its
 // first token, and a sequence's tiles past its own keys are left unwritten.
 // ------------------------------------------------------------------------------------------------
@@ -300,81 +284,74 @@ __device__ __forceinline__ VTile v_tile(const VQuantArgs& a, int64_t item) {
 }
 
 template <int D, int DT, bool NVF>
-__global__ void __launch_bounds__(256) quant_v_kernel(VQuantArgs a, int64_t items) {
-  __shared__ float tile[64][D + 1];
-  constexpr int VEC_PER_ROW = D / 8;             // 8 values per load
-  constexpr int NVEC = 64 * VEC_PER_ROW / 256;   // loads per thread and tile
+__global__ void __launch_bounds__(D) quant_v_kernel(VQuantArgs a) {
+  constexpr int ES = DT == kBF16 ? 2 : 4;  // bytes per element
+  constexpr int ROW = D * ES;              // bytes per key row
+  __shared__ __align__(16) uint8_t tile[64 * ROW];
   const int t = threadIdx.x;
-  float nxt[NVEC][8];
-  auto load_tile = [&](const VTile& vt) {
+  const VTile vt = v_tile(a, blockIdx.x);
+  if (!vt.ok) return;  // the whole block
+  const int j = vt.j;
 #pragma unroll
-    for (int u = 0; u < NVEC; u++) {
-      const int idx = t + 256 * u, row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
-      const int tok = vt.j * 64 + row;
-      const bool valid = vt.ok && tok < vt.N;
-      load8<DT>(a.v, (vt.src_row0 + (valid ? tok : 0) * vt.src_stride) * D + cv * 8, valid, nxt[u]);
+  for (int idx = t; idx < 64 * ROW / 16; idx += D) {
+    const int row = idx / (ROW / 16), chunk = idx % (ROW / 16);
+    const int tok = j * 64 + row;
+    const bool valid = tok < vt.N;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.v) +
+                         (vt.src_row0 + (int64_t)(valid ? tok : 0) * vt.src_stride) * ROW + chunk * 16;
+    cp_async16(smem_u32(tile + row * ROW + chunk * 16), src, valid ? 16u : 0u);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  const int p = t % (D / 2), h = t / (D / 2);
+  float x[2][32];  // channels 2p, 2p+1 over keys 32h..32h+31
+#pragma unroll
+  for (int i = 0; i < 32; i++) {
+    const uint8_t* r = tile + (32 * h + i) * ROW;
+    if (DT == kBF16) {
+      const uint32_t wv = *reinterpret_cast<const uint32_t*>(r + 4 * p);
+      x[0][i] = __uint_as_float(wv << 16);
+      x[1][i] = __uint_as_float(wv & 0xFFFF0000u);
+    } else {
+      const float2 f = *reinterpret_cast<const float2*>(r + 8 * p);
+      x[0][i] = f.x;
+      x[1][i] = f.y;
     }
-  };
-  int64_t item = blockIdx.x;
-  VTile next = v_tile(a, item);
-  load_tile(next);
-  for (; item < items; item += gridDim.x) {
-    __syncthreads();  // the previous tile has been read out of shared memory
+  }
 #pragma unroll
-    for (int u = 0; u < NVEC; u++) {
-      const int idx = t + 256 * u, row = idx / VEC_PER_ROW, cv = idx % VEC_PER_ROW;
-#pragma unroll
-      for (int i = 0; i < 8; i++) tile[row][cv * 8 + i] = nxt[u][i];
-    }
-    const VTile me = next;
-    if (item + gridDim.x < items) {
-      next = v_tile(a, item + gridDim.x);
-      load_tile(next);  // in flight while this tile is quantized
-    }
-    __syncthreads();
-    if (!me.ok) continue;
-    const int j = me.j;
-    for (int it = t; it < 2 * D; it += 256) {
-      const int c = it % D, h = it / D;
-      if (NVF) {
-        // two blocks of 16 keys; one scale atom per 64-key tile, keys 16b..16b+15 in byte b of
-        // channel c's word
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 32; i++) x[i] = tile[h * 32 + i][c];
-        uint32_t w[4];
-        const uint32_t b = nvfp4_block(x, w) | (nvfp4_block(x + 16, w + 2) << 8);
-        uint8_t* dst = a.v_codes + (me.vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-        uint8_t* atom = a.v_scales + me.vtile * 512;
-        *reinterpret_cast<uint16_t*>(atom + (c % 32) * 16 + (c / 32) * 4 + 2 * h) = (uint16_t)b;
-        if (D == 64) *reinterpret_cast<uint16_t*>(atom + ((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 * h) = 0;
-        continue;
-      }
-      float amax = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(tile[h * 32 + i][c]));
-      const int e = shared_exponent(amax, a.rule);
-      const float inv = pow2_neg(e);
-      uint32_t w[4];
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const int b = h * 32 + q * 8;
-        w[q] = cvt_e2m1x8(__fmul_rn(tile[b + 0][c], inv), __fmul_rn(tile[b + 1][c], inv),
-                          __fmul_rn(tile[b + 2][c], inv), __fmul_rn(tile[b + 3][c], inv),
-                          __fmul_rn(tile[b + 4][c], inv), __fmul_rn(tile[b + 5][c], inv),
-                          __fmul_rn(tile[b + 6][c], inv), __fmul_rn(tile[b + 7][c], inv));
-      }
-      uint8_t* dst = a.v_codes + (me.vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+  for (int k = 0; k < 2; k++) {
+    const int c = 2 * p + k;
+    const float* v = x[k];
+    uint8_t* dst = a.v_codes + (vt.vtile * D + c) * 32 + ((h ^ ((c >> 2) & 1)) * 16);
+    uint32_t w[4];
+    if (NVF) {
+      // two blocks of 16 keys; one scale atom per 64-key tile, keys 16b..16b+15 in byte b of
+      // channel c's word
+      const uint32_t b = nvfp4_block(v, w) | (nvfp4_block(v + 16, w + 2) << 8);
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-      uint8_t* atom = a.v_scales + me.atom_tile * 512;
-      atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
-      if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
-      // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
-      if (j == me.T64 - 1 && (j % 2) == 0) {
-        atom[(c % 32) * 16 + (c / 32) * 4 + 2 + h] = 0;
-        if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 + h] = 0;
-      }
+      uint8_t* atom = a.v_scales + vt.vtile * 512;
+      *reinterpret_cast<uint16_t*>(atom + (c % 32) * 16 + (c / 32) * 4 + 2 * h) = (uint16_t)b;
+      if (D == 64) *reinterpret_cast<uint16_t*>(atom + ((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 * h) = 0;
+      continue;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = shared_exponent(amax, a.rule);
+    const float inv = pow2_neg(e);
+#pragma unroll
+    for (int q = 0; q < 4; q++)
+      w[q] = cvt_e2m1x8(__fmul_rn(v[8 * q + 0], inv), __fmul_rn(v[8 * q + 1], inv), __fmul_rn(v[8 * q + 2], inv),
+                        __fmul_rn(v[8 * q + 3], inv), __fmul_rn(v[8 * q + 4], inv), __fmul_rn(v[8 * q + 5], inv),
+                        __fmul_rn(v[8 * q + 6], inv), __fmul_rn(v[8 * q + 7], inv));
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    uint8_t* atom = a.v_scales + vt.atom_tile * 512;
+    atom[(c % 32) * 16 + (c / 32) * 4 + (j % 2) * 2 + h] = (uint8_t)(e + 127);
+    if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + (j % 2) * 2 + h] = 0;
+    // a ragged last 64-key tile that is the even half of its atom leaves the odd half unwritten
+    if (j == vt.T64 - 1 && (j % 2) == 0) {
+      atom[(c % 32) * 16 + (c / 32) * 4 + 2 + h] = 0;
+      if (D == 64) atom[((c + 64) % 32) * 16 + ((c + 64) / 32) * 4 + 2 + h] = 0;
     }
   }
 }
@@ -435,18 +412,17 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(PlainQuantArgs a) {
 // ------------------------------------------------------------------------------------------------
 template <int D, int DT>
 static void qk_launch(const QKQuantArgs& a, dim3 grid, cudaStream_t s) {
-  if (a.fmt == kFmtNVFP4) rotate_quant_qk_kernel<D, DT, true><<<grid, 256, 0, s>>>(a);
-  else rotate_quant_qk_kernel<D, DT, false><<<grid, 256, 0, s>>>(a);
+  constexpr int T = QKBlock<D, DT>::ROWS;
+  if (a.fmt == kFmtNVFP4) rotate_quant_qk_kernel<D, DT, true><<<grid, T, 0, s>>>(a);
+  else rotate_quant_qk_kernel<D, DT, false><<<grid, T, 0, s>>>(a);
 }
 
 cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaStream_t s) {
-  const int64_t rows = a.vl.cu_seqlens != nullptr ? (int64_t)a.BH * a.vl.tiles_per_head * 128
-                                                  : (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128) * 128;
-  const int rows_per_block = 256 / (D / 32);
-  // enough blocks for every SM to hold several at once; each loops over the rest of the rows
-  const int64_t want = (rows + rows_per_block - 1) / rows_per_block;
-  constexpr int64_t kMaxBlocks = 148 * 8;
-  dim3 grid((unsigned)(want < kMaxBlocks ? want : kMaxBlocks), 2);
+  // one block per 128-row packed tile or part of one, over the longer of Q and K
+  const int64_t tiles = a.vl.cu_seqlens != nullptr ? (int64_t)a.BH * a.vl.tiles_per_head
+                                                   : (int64_t)a.BH * (((a.N > a.Nk ? a.N : a.Nk) + 127) / 128);
+  const int split = dtype == kBF16 ? QKBlock<128, kBF16>::SPLIT : QKBlock<128, kFP32>::SPLIT;
+  const dim3 grid((unsigned)(tiles * split), 2);
   if (D == 128 && dtype == kBF16) qk_launch<128, kBF16>(a, grid, s);
   else if (D == 128) qk_launch<128, kFP32>(a, grid, s);
   else if (dtype == kBF16) qk_launch<64, kBF16>(a, grid, s);
@@ -456,11 +432,9 @@ cudaError_t launch_rotate_quant_qk(const QKQuantArgs& a, int D, int dtype, cudaS
 
 template <int D, int DT>
 static void v_launch(const VQuantArgs& a, int64_t items, cudaStream_t s) {
-  // several blocks per SM (33 KB of shared memory each at D = 128), each striding over the items
-  constexpr int64_t kMaxBlocks = 148 * 6;
-  const unsigned blocks = (unsigned)(items < kMaxBlocks ? items : kMaxBlocks);
-  if (a.fmt == kFmtNVFP4) quant_v_kernel<D, DT, true><<<blocks, 256, 0, s>>>(a, items);
-  else quant_v_kernel<D, DT, false><<<blocks, 256, 0, s>>>(a, items);
+  // one block of D threads per item (16 or 32 KB of shared memory at D = 128)
+  if (a.fmt == kFmtNVFP4) quant_v_kernel<D, DT, true><<<(unsigned)items, D, 0, s>>>(a);
+  else quant_v_kernel<D, DT, false><<<(unsigned)items, D, 0, s>>>(a);
 }
 
 cudaError_t launch_quant_v(const VQuantArgs& a, int D, int dtype, cudaStream_t s) {
