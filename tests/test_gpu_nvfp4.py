@@ -5,9 +5,8 @@ scales, against the oracle's NVFP4 functions.
    extreme magnitudes), the rotated Q/K operands and the key-major V operand.  Both sides divide
    by the scale in fp32 with one rounding and round the quotient to E2M1 the same way.
 2. The attention kernel (tcgen05 kind::mxf4nvf4, block16, UE4M3 scales) against the oracle's NVFP4
-   attention: rel-L2 <= 2e-3 and max-abs <= 2e-2 (units of V ~ N(0, 1)), with the per-row allowance
-   for one P^ code flip (the kernel takes P~ / scale as one exp2, the oracle divides fl32(P~ * 2688)
-   by the scale, so an occasional code lands on the other side of a rounding boundary).
+   attention: rel-L2 <= 2e-3 and max-abs <= 2e-2 (units of V ~ N(0, 1)), each case's largest
+   deviation printed as a DIAG line.
 3. Error against exact fp32 attention of NVFP4 beside MXFP4 (UOS) on the outlier workload: printed
    as DIAG lines (run with -s)."""
 import json
@@ -102,13 +101,13 @@ def test_attention_matches_the_oracle(BH, N, d, dtype, pnq, tau):
     res = oracle.forward_rows(q, k, v, rows, scale, pnq=pnq, tau=tau, fmt=oracle.FMT_NVFP4)
     ref = oracle.round_to_bf16(res["out"]) if dtype == "bf16" else res["out"].astype(np.float32).astype(np.float64)
     got = got[:, rows]
-    # one P^ flip moves a row by at most 2 * (largest P^ step) * max|V^| / l; the largest step of
-    # a block is 1/6 of its scale range: 2 * 448 / 2688 = 1/3 of the running max's unit
-    tol = MAX_ABS_TOL + (2 / 3) * 1.1 * float(np.abs(v).max()) / res["l"][:, :, None]
     e = rel_l2(got, ref)
+    dev = np.abs(got - ref)
+    print("DIAG " + json.dumps({"diag": "nvfp4_parity", "BH": BH, "N": N, "d": d, "dtype": dtype, "pnq": pnq,
+                                "tau": tau, "rel_l2": e, "max_abs": float(dev.max()),
+                                "elements_over_2e-2": int((dev > MAX_ABS_TOL).sum())}))
     assert np.isfinite(got).all()
-    assert e <= REL_L2_TOL and bool(np.all(np.abs(got - ref) <= tol)), \
-        f"rel_l2={e:.3e} max_abs={float(np.max(np.abs(got - ref))):.3e}"
+    assert e <= REL_L2_TOL and float(dev.max()) <= MAX_ABS_TOL, f"rel_l2={e:.3e} max_abs={float(dev.max()):.3e}"
 
 
 def test_error_against_exact_attention_nvfp4_vs_mxfp4():
@@ -146,8 +145,10 @@ def test_nvfp4_cross_and_host_paths():
     res = oracle.forward_rows(q, k, v, np.arange(300), scale, tau=8.0, fmt=oracle.FMT_NVFP4)
     ref = oracle.round_to_bf16(res["out"])
     got = out_to_numpy(out)[0]
-    tol = MAX_ABS_TOL + (2 / 3) * 1.1 * float(np.abs(v).max()) / res["l"][:, :, None]
-    assert rel_l2(got, ref) <= REL_L2_TOL and bool(np.all(np.abs(got - ref) <= tol))
+    dev_abs = float(np.max(np.abs(got - ref)))
+    print("DIAG " + json.dumps({"diag": "nvfp4_parity", "case": "cross 300 x 1000", "rel_l2": rel_l2(got, ref),
+                                "max_abs": dev_abs}))
+    assert rel_l2(got, ref) <= REL_L2_TOL and dev_abs <= MAX_ABS_TOL
 
     qs, ks, vs = (_dev(x, "bf16") for x in _draw(6, 1000, 128, "bf16", seed=43))
     dev = binding.mxattn_forward(qs, ks, vs, 0.088, NV)

@@ -1,12 +1,14 @@
 """Packed batches of variable-length sequences (mxattn_forward_varlen): token-major [T, H, d] inputs,
 device cu_seqlens.  Every sequence is an attention problem of its own, so the oracle runs each one
-alone (oracle.forward_varlen) and the comparison is element by element: rel-L2 <= 2e-3 over the
-batch, and per element max-abs <= 2e-2 in units of V ~ N(0, 1), widened for rows with a small row
-sum l to what one P^ code flip moves (see _flip_bound): short sequences have rows of a few keys,
-where one exp2 rounding that lands a P~ value on the other side of an E2M1 boundary is visible.
+alone (oracle.forward_varlen) and the comparison is element by element at the plain bound:
+rel-L2 <= 2e-3 over the batch and max-abs <= 2e-2 per element, in units of V ~ N(0, 1), short
+sequences (rows of a few keys, where one flipped P^ code would be visible) included.  Each case
+prints a DIAG line with its largest deviation (run with -s).
 Bit-exact checks tie the packing to the fixed-length kernels: every sequence equals mxattn_forward
 run on it alone, a single sequence equals mxattn_forward on [1, H, N, d], and equal-length
 sequences equal mxattn_forward with B = nseq."""
+import json
+
 import numpy as np
 import pytest
 
@@ -39,20 +41,13 @@ def _cu(lengths):
     return cu, torch.from_numpy(cu).cuda()
 
 
-def _check(got, ref, l=None, vmax=None):
+def _check(got, ref, case):
     assert np.isfinite(got).all()
-    e, m = rel_l2(got, ref), float(np.max(np.abs(got - ref)))
-    tol = MAX_ABS_TOL if l is None else _flip_bound(l, vmax)[:, :, None]
-    assert e <= REL_L2_TOL and bool(np.all(np.abs(got - ref) <= tol)), f"rel_l2={e:.3e} max_abs={m:.3e}"
-
-
-def _flip_bound(l, vmax):
-    """Per-row max-abs tolerance: 2e-2 plus what one P^ code flip can move.  P~ <= 1 puts every
-    group's scale at 2^-2 or below (UOS: the block max maps into (3.625, 7.25]), where neighbouring
-    E2M1 codes up to 4 are at most 1 apart: a flip moves one P^ value by <= 2^-2, hence the output
-    row sum(P^ V^) / l by <= 2^-2 (|V^| + |O|) / l <= 2 * 2^-2 * max|V^| / l (under PNQ l moves with
-    it).  max|V^| <= 4/3.625 max|V| (a block max scaled into (3.625, 7.25] rounds up to 4 at most)."""
-    return MAX_ABS_TOL + 0.5 * vmax / l
+    e = rel_l2(got, ref)
+    dev = np.abs(got - ref)
+    print("DIAG " + json.dumps({"diag": "varlen_parity", "case": case, "rel_l2": e, "max_abs": float(dev.max()),
+                                "elements_over_2e-2": int((dev > MAX_ABS_TOL).sum())}))
+    assert e <= REL_L2_TOL and float(dev.max()) <= MAX_ABS_TOL, f"rel_l2={e:.3e} max_abs={float(dev.max()):.3e}"
 
 
 @pytest.mark.parametrize("lengths,H,d,dtype", [
@@ -78,10 +73,9 @@ def test_varlen_matches_the_oracle(lengths, H, d, dtype, pnq, causal):
                                         workspace=ws)
     torch.cuda.synchronize()
     assert binding.mxattn_get_device_error(ws) == 0
-    ref, l = oracle.forward_varlen(q, k, v, cu, np.arange(T), scale, pnq=pnq, tau=8.0, causal=causal,
-                                   with_l=True)
+    ref = oracle.forward_varlen(q, k, v, cu, np.arange(T), scale, pnq=pnq, tau=8.0, causal=causal)
     ref = oracle.round_to_bf16(ref) if dtype == "bf16" else ref.astype(np.float32).astype(np.float64)
-    _check(out_to_numpy(out), ref, l, 4 / 3.625 * float(np.abs(v).max()))
+    _check(out_to_numpy(out), ref, f"lengths={lengths} H={H} d={d} {dtype} pnq={pnq} causal={causal}")
 
     # each sequence on its own through the fixed-length pass: the same bits
     got = out.view(torch.int16 if dtype == "bf16" else torch.int32)
@@ -132,7 +126,7 @@ def test_video_mix_sampled_rows():
     torch.cuda.synchronize()
     rows = np.unique(np.concatenate([cu[s] + inputs.sample_rows(n, 8) for s, n in enumerate(lengths)]))
     ref = oracle.round_to_bf16(oracle.forward_varlen(q, k, v, cu, rows, 0.088, tau=8.0))
-    _check(out_to_numpy(out)[rows], ref)
+    _check(out_to_numpy(out)[rows], ref, "video mix sampled rows")
 
 
 @pytest.mark.parametrize("table", [[0, 50, 40, 100], [0, 50, 100, 120], [3, 50, 80, 100]])
