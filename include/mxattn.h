@@ -129,7 +129,10 @@ typedef struct mxattn_opts {
   int pnq;                 /* 1: l from the quantized tile (PNQ); 0: direct placement   */
   int rotate;              /* 1: Hadamard-rotate Q and K before quantizing               */
   int dtype;               /* mxattn_dtype of q, k, v, out                               */
-  int key_tile;            /* keys per online-softmax step; 64 is supported             */
+  int key_tile;            /* keys per online-softmax step: 128 (the default, the       */
+                           /* faster kernel) or 64; NVFP4 runs only with 64 (128 with   */
+                           /* NVFP4 returns MXATTN_ERR_UNSUPPORTED).  The lazy running   */
+                           /* max moves at tile boundaries, so results depend on it.     */
   float rescale_tau;       /* the running max moves only when it grows by more than    */
                            /* tau (log2 units); 0 = eager FlashAttention-2 update       */
   void* workspace;         /* device buffer, see mxattn_workspace_bytes                  */
@@ -151,8 +154,8 @@ typedef struct mxattn_opts {
 } mxattn_opts;
 
 /* Fill *opts with the defaults: UOS, qmax 7.25, pnq 1, rotate 1, bf16,
- * key_tile 64, rescale_tau 8, no workspace, default wait budget, MXFP4,
- * causal 0. */
+ * key_tile 128, rescale_tau 8, no workspace, default wait budget, MXFP4,
+ * causal 0.  (NVFP4 callers set key_tile = 64.) */
 MXATTN_API void mxattn_opts_default(mxattn_opts* opts);
 
 /* Bytes of workspace mxattn_forward needs for this problem (status block plus

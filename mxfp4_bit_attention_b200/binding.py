@@ -53,7 +53,7 @@ class Opts:
     qmax: float = 7.25
     pnq: bool = True
     rotate: bool = True
-    key_tile: int = 64
+    key_tile: int = 128  # 64 for the NVFP4 comparison format
     rescale_tau: float = 8.0
     wait_budget_cycles: int = 0  # 0: the library's default (about one second)
     causal: bool = False  # self-attention: query row i sees keys 0..i
@@ -228,7 +228,7 @@ def mxattn_attention_mxfp4(ops, B, H, N, d, softmax_scale, out, opts: Opts | Non
     return out
 
 
-def dump_layout(N: int, d: int, key_tile: int = 64) -> dict:
+def dump_layout(N: int, d: int, key_tile: int = 128) -> dict:
     """Byte offsets of the diagnostic dump for key tiles of key_tile keys (mirrors the header)."""
     KT = key_tile
     T = (N + KT - 1) // KT

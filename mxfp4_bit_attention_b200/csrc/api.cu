@@ -119,7 +119,7 @@ void mxattn_opts_default(mxattn_opts* o) {
   o->pnq = 1;
   o->rotate = 1;
   o->dtype = MXATTN_BF16;
-  o->key_tile = 64;
+  o->key_tile = 128;
   o->rescale_tau = 8.0f;
   o->workspace = nullptr;
   o->workspace_bytes = 0;

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(lib):
 def test_host_only_calls(lib):
     o = binding.COpts()
     lib.mxattn_opts_default(ctypes.byref(o))
-    assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 64)
+    assert (o.scale_rule, o.pnq, o.rotate, o.key_tile) == (0, 1, 1, 128)
     assert abs(o.qmax - 7.25) < 1e-7 and abs(o.rescale_tau - 8.0) < 1e-7
     assert o.wait_budget_cycles == 0  # the library's default budget
     assert o.causal == 0 and o.format == 0

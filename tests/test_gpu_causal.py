@@ -33,8 +33,8 @@ def _dev(x, dtype):
     return (t.to(torch.bfloat16) if dtype == "bf16" else t)[None]  # exact: the values are bf16 already
 
 
-def _ref(q, k, v, rows, scale, dtype, pnq=True, tau=8.0):
-    ref = oracle.forward_rows(q, k, v, rows, scale, pnq=pnq, tau=tau, causal=True)["out"]
+def _ref(q, k, v, rows, scale, dtype, pnq=True, tau=8.0, kt=128):
+    ref = oracle.forward_rows(q, k, v, rows, scale, pnq=pnq, tau=tau, causal=True, key_tile=kt)["out"]
     return oracle.round_to_bf16(ref) if dtype == "bf16" else ref.astype(np.float32).astype(np.float64)
 
 
@@ -53,14 +53,15 @@ def _check(got, ref):
     (1, 777, 64, "bf16"),     # ragged, d = 64
 ])
 @pytest.mark.parametrize("pnq", [True, False])
-def test_causal_matches_the_oracle(BH, N, d, dtype, pnq):
+@pytest.mark.parametrize("kt", [64, 128])
+def test_causal_matches_the_oracle(BH, N, d, dtype, pnq, kt):
     import torch
     q, k, v = _draw(BH, N, d, dtype, seed=500 + N + d)
     scale = float(np.float32(d ** -0.5))
     out = binding.mxattn_forward(_dev(q, dtype), _dev(k, dtype), _dev(v, dtype), scale,
-                                 binding.Opts(pnq=pnq, causal=True))
+                                 binding.Opts(pnq=pnq, causal=True, key_tile=kt))
     torch.cuda.synchronize()
-    _check(out_to_numpy(out)[0], _ref(q, k, v, np.arange(N), scale, dtype, pnq=pnq))
+    _check(out_to_numpy(out)[0], _ref(q, k, v, np.arange(N), scale, dtype, pnq=pnq, kt=kt))
 
 
 def test_causal_first_row_is_the_quantized_first_value_row():
@@ -75,20 +76,21 @@ def test_causal_first_row_is_the_quantized_first_value_row():
     np.testing.assert_array_equal(out_to_numpy(out)[0, 0, 0], vhat[:, 0])
 
 
-def test_causal_outlier_sampled_rows_and_repeat():
+@pytest.mark.parametrize("kt", [64, 128])
+def test_causal_outlier_sampled_rows_and_repeat(kt):
     import torch
     w = inputs.WORKLOADS["outlier"]
     g = inputs.generate(w, heads=[0, 5])
     q, k, v = (to_device(g[n], w.dtype, (1, 2, w.N, w.d)) for n in "qkv")
     scale = float(np.float32(w.d ** -0.5))
-    opts = binding.Opts(causal=True)
+    opts = binding.Opts(causal=True, key_tile=kt)
     out = binding.mxattn_forward(q, k, v, scale, opts)
     again = binding.mxattn_forward(q, k, v, scale, opts)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), again.view(torch.int16))
     rows = np.unique(np.concatenate([inputs.sample_rows(w.N, 24), [127, 128, 255, 256, 2047, 2048, 4095]]))
     qf, kf, vf = (inputs.as_fp32(g[n], w.dtype) for n in "qkv")
-    _check(out_to_numpy(out)[0][:, rows], _ref(qf, kf, vf, rows, scale, "bf16"))
+    _check(out_to_numpy(out)[0][:, rows], _ref(qf, kf, vf, rows, scale, "bf16", kt=kt))
 
 
 def test_causal_720p_sampled_rows():

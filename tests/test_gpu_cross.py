@@ -37,15 +37,16 @@ def _dev(x, dtype):
     (3, 200, 64, 64, "bf16"),      # exactly one key tile
 ])
 @pytest.mark.parametrize("pnq", [True, False])
-def test_cross_attention_matches_the_oracle(BH, Nq, Nk, d, dtype, pnq):
+@pytest.mark.parametrize("kt", [64, 128])
+def test_cross_attention_matches_the_oracle(BH, Nq, Nk, d, dtype, pnq, kt):
     import torch
     q, k, v = _draw(BH, Nq, Nk, d, dtype, seed=1000 + Nq + Nk + d)
     scale = float(np.float32(d ** -0.5))
-    opts = binding.Opts(pnq=pnq)
+    opts = binding.Opts(pnq=pnq, key_tile=kt)
     out = binding.mxattn_forward_cross(_dev(q, dtype), _dev(k, dtype), _dev(v, dtype), scale, opts)
     torch.cuda.synchronize()
     got = out_to_numpy(out)[0]
-    ref = oracle.forward_rows(q, k, v, np.arange(Nq), scale, pnq=pnq, tau=8.0)["out"]
+    ref = oracle.forward_rows(q, k, v, np.arange(Nq), scale, pnq=pnq, tau=8.0, key_tile=kt)["out"]
     ref = oracle.round_to_bf16(ref) if dtype == "bf16" else ref.astype(np.float32).astype(np.float64)
     assert np.isfinite(got).all()
     e, m = rel_l2(got, ref), float(np.max(np.abs(got - ref)))
@@ -74,5 +75,5 @@ def test_video_to_text_cross_attention_sampled():
     torch.cuda.synchronize()
     rows = inputs.sample_rows(Nq, 32)
     got = out_to_numpy(out)[0][:, rows]
-    ref = oracle.round_to_bf16(oracle.forward_rows(q, k, v, rows, scale, tau=8.0)["out"])
+    ref = oracle.round_to_bf16(oracle.forward_rows(q, k, v, rows, scale, tau=8.0, key_tile=128)["out"])
     assert rel_l2(got, ref) <= REL_L2_TOL and float(np.max(np.abs(got - ref))) <= MAX_ABS_TOL

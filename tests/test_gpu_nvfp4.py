@@ -21,7 +21,7 @@ from helpers import MAX_ABS_TOL, REL_L2_TOL, out_to_numpy, rel_l2, to_device
 
 pytestmark = pytest.mark.gpu
 
-NV = binding.Opts(format=binding.FMT_NVFP4)
+NV = binding.Opts(format=binding.FMT_NVFP4, key_tile=64)  # NVFP4 runs with 64-key tiles
 
 
 @pytest.mark.parametrize("axis", [0, 1])
@@ -93,7 +93,7 @@ def test_attention_matches_the_oracle(BH, N, d, dtype, pnq, tau):
     import torch
     q, k, v = _draw(BH, N, d, dtype, seed=900 + N + d)
     scale = float(np.float32(d ** -0.5))
-    opts = binding.Opts(format=binding.FMT_NVFP4, pnq=pnq, rescale_tau=tau)
+    opts = binding.Opts(format=binding.FMT_NVFP4, pnq=pnq, rescale_tau=tau, key_tile=64)
     out = binding.mxattn_forward(_dev(q, dtype), _dev(k, dtype), _dev(v, dtype), scale, opts)
     torch.cuda.synchronize()
     got = out_to_numpy(out)[0]
@@ -123,7 +123,8 @@ def test_error_against_exact_attention_nvfp4_vs_mxfp4():
     for label, fmt in (("MXFP4 UOS", binding.FMT_MXFP4), ("NVFP4", binding.FMT_NVFP4)):
         for tau in (0.0, 8.0):
             for pnq in (True, False):
-                out = binding.mxattn_forward(q, k, v, scale, binding.Opts(format=fmt, pnq=pnq, rescale_tau=tau)).float()
+                opts = binding.Opts(format=fmt, pnq=pnq, rescale_tau=tau, key_tile=64)
+                out = binding.mxattn_forward(q, k, v, scale, opts).float()
                 err = (out - exact).double()
                 rel = float(err.norm() / exact.double().norm())
                 table[(label, tau, pnq)] = rel
@@ -162,4 +163,4 @@ def test_nvfp4_cross_and_host_paths():
 def test_nvfp4_rejects_masking():
     q, k, v = (_dev(x, "fp32") for x in _draw(1, 128, 64, "fp32", seed=2))
     with pytest.raises(binding.MXAttnError):
-        binding.mxattn_forward(q, k, v, 0.125, binding.Opts(format=binding.FMT_NVFP4, causal=True))
+        binding.mxattn_forward(q, k, v, 0.125, binding.Opts(format=binding.FMT_NVFP4, causal=True, key_tile=64))

@@ -59,13 +59,14 @@ def _check(got, ref, case):
 ])
 @pytest.mark.parametrize("pnq", [True, False])
 @pytest.mark.parametrize("causal", [False, True])
-def test_varlen_matches_the_oracle(lengths, H, d, dtype, pnq, causal):
+@pytest.mark.parametrize("kt", [64, 128])
+def test_varlen_matches_the_oracle(lengths, H, d, dtype, pnq, causal, kt):
     import torch
     cu, cu_dev = _cu(lengths)
     T = int(cu[-1])
     q, k, v = _draw(T, H, d, dtype, seed=700 + T + d)
     scale = float(np.float32(d ** -0.5))
-    opts = binding.Opts(pnq=pnq, causal=causal)
+    opts = binding.Opts(pnq=pnq, causal=causal, key_tile=kt)
     ws = torch.zeros(binding.load().mxattn_workspace_bytes_varlen(
         len(lengths), H, T, d, binding.ctypes.byref(binding._copts(opts, binding._dtype_code(_dev(q[:1], dtype))))),
         dtype=torch.uint8, device="cuda")
@@ -73,9 +74,9 @@ def test_varlen_matches_the_oracle(lengths, H, d, dtype, pnq, causal):
                                         workspace=ws)
     torch.cuda.synchronize()
     assert binding.mxattn_get_device_error(ws) == 0
-    ref = oracle.forward_varlen(q, k, v, cu, np.arange(T), scale, pnq=pnq, tau=8.0, causal=causal)
+    ref = oracle.forward_varlen(q, k, v, cu, np.arange(T), scale, pnq=pnq, tau=8.0, causal=causal, key_tile=kt)
     ref = oracle.round_to_bf16(ref) if dtype == "bf16" else ref.astype(np.float32).astype(np.float64)
-    _check(out_to_numpy(out), ref, f"lengths={lengths} H={H} d={d} {dtype} pnq={pnq} causal={causal}")
+    _check(out_to_numpy(out), ref, f"lengths={lengths} H={H} d={d} {dtype} pnq={pnq} causal={causal} kt={kt}")
 
     # each sequence on its own through the fixed-length pass: the same bits
     got = out.view(torch.int16 if dtype == "bf16" else torch.int32)
@@ -125,7 +126,7 @@ def test_video_mix_sampled_rows():
     out = binding.mxattn_forward_varlen(_dev(q, "bf16"), _dev(k, "bf16"), _dev(v, "bf16"), cu_dev, 0.088)
     torch.cuda.synchronize()
     rows = np.unique(np.concatenate([cu[s] + inputs.sample_rows(n, 8) for s, n in enumerate(lengths)]))
-    ref = oracle.round_to_bf16(oracle.forward_varlen(q, k, v, cu, rows, 0.088, tau=8.0))
+    ref = oracle.round_to_bf16(oracle.forward_varlen(q, k, v, cu, rows, 0.088, tau=8.0, key_tile=128))
     _check(out_to_numpy(out)[rows], ref, "video mix sampled rows")
 
 
