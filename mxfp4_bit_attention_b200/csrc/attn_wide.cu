@@ -479,6 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       // exp(0) is in the oracle.
       uint32_t eb[4], w[16];
       float psum[4];
+      // P buffer j % 4 was last read by PV(j-4), which the QK issuer saw complete before it
+      // committed S(j).  Codes in the MMA's 64-byte swizzled rows: group g (16 bytes) at chunk
+      // g ^ ((row >> 1) & 3); the four scale bytes in the row's word of the scale atom.  Each
+      // piece is stored as soon as it exists, so the stores overlap the rest of the code phase.
+      const int pb = j % kPBufs;
+      uint8_t* prow = smem + L::P_CODES + pb * L::P_BYTES + row * 64;
+      const int sw = (row >> 1) & 3;
       auto codes = [&](float fr) {
         float ex[4];  // the groups' shared exponents e
 #pragma unroll
@@ -486,10 +493,19 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
           ex[g] = shared_exponent_log2f_rule<FLOOR>((gmax[g] - fr) * c, log2q, eb[g]);
           psum[g] = 0.f;
         }
+        *reinterpret_cast<uint32_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
+            eb[0] | (eb[1] << 8) | (eb[2] << 16) | (eb[3] << 24);
+        auto store = [&](int g) {
+          *reinterpret_cast<uint4*>(prow + ((g ^ sw) * 16)) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+        };
         group_codes<0, PNQ>(s, fr, c, ex[0], w, psum[0]);
+        store(0);
         group_codes<1, PNQ>(s, fr, c, ex[1], w + 4, psum[1]);
+        store(1);
         group_codes<2, PNQ>(s, fr, c, ex[2], w + 8, psum[2]);
+        store(2);
         group_codes<3, PNQ>(s, fr, c, ex[3], w + 12, psum[3]);
+        store(3);
       };
       // The running max before this tile is the one after tile j-1, which the other group hands
       // over through shared memory (its XCH barrier); the codes are formed in the frame after this
@@ -554,17 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         }
         tmem_wait_st();
       }
-      // P buffer j % 4 was last read by PV(j-4), which the QK issuer saw complete before it
-      // committed S(j).  Codes in the MMA's 64-byte swizzled rows: group g (16 bytes) at chunk
-      // g ^ ((row >> 1) & 3); the four scale bytes in the row's word of the scale atom.
-      const int pb = j % kPBufs;
-      uint8_t* prow = smem + L::P_CODES + pb * L::P_BYTES + row * 64;
-      const int sw = (row >> 1) & 3;
-#pragma unroll
-      for (int g = 0; g < 4; g++)
-        *reinterpret_cast<uint4*>(prow + ((g ^ sw) * 16)) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-      *reinterpret_cast<uint32_t*>(smem + L::SF_P + pb * 512 + (row % 32) * 16 + (row / 32) * 4) =
-          eb[0] | (eb[1] << 8) | (eb[2] << 16) | (eb[3] << 24);
+      // the P codes and scales of this tile are in shared memory (stored by codes())
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
