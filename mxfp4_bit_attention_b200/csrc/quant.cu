@@ -21,15 +21,25 @@ namespace mxattn {
 // One NVFP4 block of 16 values (the comparison format): the scale is the E4M3 rounding of
 // fl32(amax / 6), each value is divided by it in fp32 (correctly rounded) and rounded to E2M1
 // with saturation; a scale that rounds to zero gives zero codes.  Returns the scale byte.
+// The quotients: with r = RN(1/s), y = RN(v r) is within an ulp of v/s, the remainder
+// v - y s is exact in one fma, and RN(y + (v - y s) r) is RN(v/s) (Markstein's theorem); three
+// FMA-pipe operations per value instead of a division (checked against RN(v/s) for every positive
+// E4M3 scale on 25 million quotients, and bit-exact against the oracle's division in the tests).
 __device__ __forceinline__ uint32_t nvfp4_block(const float* v, uint32_t* w) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; i++) amax = fmaxf(amax, fabsf(v[i]));
   const uint32_t byte = cvt_e4m3x2(__fdiv_rn(amax, 6.f), 0.f) & 0xFFu;
   const float s = e4m3x2_to_float2(byte).x;
+  const float r = s > 0.f ? __frcp_rn(s) : 0.f;
   float y[16];
 #pragma unroll
-  for (int i = 0; i < 16; i++) y[i] = s > 0.f ? __fdiv_rn(v[i], s) : 0.f;
+  for (int i = 0; i < 16; i++) {
+    // on |v|, the sign copied back (RN is symmetric; -0 keeps its sign, as the division does)
+    const float av = fabsf(v[i]);
+    const float y0 = __fmul_rn(av, r);
+    y[i] = s > 0.f ? copysignf(__fmaf_rn(__fmaf_rn(-y0, s, av), r, y0), v[i]) : 0.f;
+  }
   w[0] = cvt_e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
   w[1] = cvt_e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
   return byte;
