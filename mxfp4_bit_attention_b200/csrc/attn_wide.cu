@@ -370,6 +370,16 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
           if (!ok) break;
           tc_fence_after();
         }
+        // V scale atom of tile j into its slot (j % 5), for PV(j): the slot was last read by PV(j-5),
+        // complete since this issuer saw PV(j-4) complete just above (or j < 5: never used).  The
+        // copy sits here, not with the PV issuer, to even out the asynchronous instructions issued
+        // per SM sub-partition; the commit below covers it, so S(j), and hence P(j), imply it.
+        if (leader) {
+          if (PNQ && D == 64)  // the ones row is B-operand row 64, inside the V atom: scale 1 for all key groups
+            *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * s + 8) = 0x7F7F7F7Fu;
+          if (PNQ && D == 64) fence_proxy_async_smem();
+          tmem_cp_sf_atom(tmem + L::T_SFV + 8 * (j % L::V_SLOTS), sb + L::SF_V + 512 * s);
+        }
         if (leader) mma_commit(bar(L::B_S_FULL + j % kSFullSlots));
         __syncwarp();
       }
@@ -392,15 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       // itself (it cannot have been refilled: that needs this warp's commit below)
       ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_KV_FULL + s), (j / kStages) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
       if (!ok) break;
-      tc_fence_after();
-      if (leader) {
-        // V scale slot f was last read by PV(j-5), complete before S(j-1) was committed, which
-        // P(j-1) arriving (seen below in the previous iteration) implies
-        if (PNQ && D == 64)  // the ones row is B-operand row 64, inside the V atom: scale 1 for all key groups
-          *reinterpret_cast<volatile uint32_t*>(smem + L::SF_V + 512 * s + 8) = 0x7F7F7F7Fu;
-        if (PNQ && D == 64) fence_proxy_async_smem();
-        tmem_cp_sf_atom(tmem + L::T_SFV + 8 * f, sb + L::SF_V + 512 * s);
-      }
+      // (the V scale atom of tile j is already in slot f: the QK issuer copied it before
+      // committing S(j))
       ok = __all_sync(0xFFFFFFFFu, mbar_wait_sleep(bar(L::B_P_FULL + pb), (j / kPBufs) & 1, abort_flag, a.wait_budget, kIssuerSleepNs));
       if (!ok) break;
       tc_fence_after();
@@ -477,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       // The codes depend on the running max after this tile (their frame).  A group's maximum is
       // taken as 2^((gmax - frame) * c): exactly 1 for the group that holds the running max, as
       // exp(0) is in the oracle.
-      uint32_t eb[4], w[16];
+      uint32_t eb[4], w[16] = {};  // (every word is set by codes() before its store)
       float psum[4];
       // P buffer j % 4 was last read by PV(j-4), which the QK issuer saw complete before it
       // committed S(j).  Codes in the MMA's 64-byte swizzled rows: group g (16 bytes) at chunk
