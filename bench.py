@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-probe", action="store_true",
+                    help="skip the dense FP4 MMA probe (the same-run peak beside the roofline's)")
     ap.add_argument("--format", default="mxfp4", choices=["mxfp4", "nvfp4"],
                     help="element format: the method's MXFP4, or the NVFP4 comparison format")
     ap.add_argument("--key-tile", type=int, default=128, choices=[64, 128],
@@ -388,6 +390,23 @@ def main():
                "call": "mxattn_forward_host"}
         del ws_host
 
+    # The dense FP4 tensor-core peak measured on this GPU in this run (mxattn_fp4_mma_probe: one CTA
+    # per SM issuing back-to-back M128 x N256 x K64 kind::mxf4 MMAs), after the timed regions.
+    probe_tflops = None
+    if not args.no_probe:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        iters, n = 100000, 256
+        binding.mxattn_fp4_mma_probe(sms, 2000, n, stream)
+        times = []
+        for _ in range(3):
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            p0.record(stream)
+            binding.mxattn_fp4_mma_probe(sms, iters, n, stream)
+            p1.record(stream)
+            torch.cuda.synchronize()
+            times.append(p0.elapsed_time(p1))
+        probe_tflops = sms * iters * 2 * 128 * n * 64 / (sorted(times)[1] * 1e-3) / 1e12
+
     fp4_peak = bf16_peak * FP4_PER_BF16
     achieved = flops / (attn_ms_max * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
@@ -398,6 +417,8 @@ def main():
                 "kernel": kernel_name(args.key_tile), "ms_per_launch": attn_ms_max,
                 "peak_source": f"{peak_kind} bf16 {bf16_peak:.1f} TFLOP/s x nominal FP4/BF16 ratio {FP4_PER_BF16:g}",
                 "frac_of_spec_9pf": achieved / 9000.0,
+                "probe_fp4_tflops": probe_tflops,
+                "frac_of_probe": None if probe_tflops is None else achieved / probe_tflops,
                 "quantizers_ms": quant_ms,
                 "quantizers_hbm_gbs": (3 * q.numel() * (q.element_size() + 0.5 + 1 / 32)) / (quant_ms * 1e-3) / 1e9}
 
