@@ -15,8 +15,9 @@
 //                      a group's next tile runs while it works on the current one; warp w and
 //                      warp w+4 own the same 32 query rows (TMEM lanes 32(w%4)..).  The running
 //                      max passes from one group to the other once per tile through shared
-//                      memory (an mbarrier per warp pair), right after the tile's max is known,
-//                      so the groups overlap everything else;
+//                      memory (one 64-bit slot per row, tagged with the tile index and polled
+//                      by the reader), right after the tile's max is known, so the groups
+//                      overlap everything else;
 //   warp 8 (one lane)  bulk-copies Q^ once and K^/V^ tiles + their scale atoms into a ring;
 //   warps 9, 10        issue S = Q^ K^T (tcgen05.mma kind::mxf4 block-scaled, M128 N128) for the
 //                      tiles of softmax group 0 and 1 respectively, so that neither group's next
@@ -97,8 +98,10 @@ struct Layout {
   static constexpr int SF_ONES = SF_P + kPBufs * 512;  // scale atom of the ones rows (constant)
   static constexpr int SF_K = SF_ONES + 512;
   static constexpr int SF_V = SF_K + kStages * 512;
-  static constexpr int MX = SF_V + kStages * 512;     // running max handed between the groups [128]
-  static constexpr int LX = MX + 512;                 // epilogue: per group l and its frame [kGroups][2][128]
+  // running max handed between the groups: per query row one 64-bit slot holding the tile index
+  // (high word) and the max after that tile (low word)
+  static constexpr int MX = SF_V + kStages * 512;
+  static constexpr int LX = MX + 8 * kBM;             // epilogue: per group l and its frame [kGroups][2][128]
   static constexpr int BARS = LX + 1024 * kGroups;
   enum {
     B_Q = 0,
@@ -108,8 +111,7 @@ struct Layout {
     B_S_FREE = B_S_FULL + kSFullSlots,  // two: one per S buffer (tile parity)
     B_P_FULL = B_S_FREE + 2,     // kPBufs
     B_O_DONE = B_P_FULL + kPBufs,  // kPBufs: PV(j) commits to O_DONE[j % kPBufs]
-    B_XCH = B_O_DONE + kPBufs,   // [source group][4 warp quadrants]: running max handed over
-    B_EPI = B_XCH + 4 * kGroups,  // every group ready for the epilogue
+    B_EPI = B_O_DONE + kPBufs,   // every group ready for the epilogue
     B_DRAIN = B_EPI + 1,
     NUM_BARS
   };
@@ -263,7 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       mbar_init(bar(L::B_P_FULL + b), 4);
       mbar_init(bar(L::B_O_DONE + b), 1);
     }
-    for (int i = 0; i < 4 * kGroups; i++) mbar_init(bar(L::B_XCH + i), 1);
     mbar_init(bar(L::B_EPI), kSoftWarps);
     mbar_init(bar(L::B_DRAIN), 3);  // one commit from each issuer
     fence_mbar_init();
@@ -281,6 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       reinterpret_cast<uint32_t*>(smem + L::SF_ONES)[i] = i == 0 ? 0x7F7F7F7Fu : 0u;
     fence_proxy_async_smem();
   }
+  for (int i = threadIdx.x; i < kBM; i += kThreads)  // no tile's index: nothing handed over yet
+    reinterpret_cast<volatile unsigned long long*>(smem + L::MX)[i] = ~0ull;
   if (warp == kQkWarp) {
     tmem_alloc(sb + L::TMEM_SLOT, kTmemCols);
     tmem_relinquish();
@@ -438,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
     const float c = a.scale_log2;
     const bool dumping = DUMP && bh == a.dump_bh && qt == a.dump_qt;
     const DumpLayout dl(D, T, kBN);
-    volatile float* mx = reinterpret_cast<volatile float*>(smem + L::MX);
+    volatile unsigned long long* mx = reinterpret_cast<volatile unsigned long long*>(smem + L::MX);
     // keys this row sees: all Nk, or under causal masking those up to its own position
     const int kmax = causal ? (qt * kBM + row + 1 < Nk ? qt * kBM + row + 1 : Nk) : Nk;
     float sm = -INFINITY;   // running max of S (raw MMA units) after this group's latest tile
@@ -511,23 +514,28 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         store(3);
       };
       // The running max before this tile is the one after tile j-1, which the other group hands
-      // over through shared memory (its XCH barrier); the codes are formed in the frame after this
-      // tile, so they wait for it.  The hand-over is published right after the maxima, before
-      // this group's own codes, so the other group's wait is short.
+      // over in the row's slot; the codes are formed in the frame after this tile, so they wait
+      // for it.  The two threads of a row write the slot in turn, each only after reading the
+      // other's value, so one slot suffices; a single 64-bit access carries the max together with
+      // its tile index, so the reader needs no barrier.  The hand-over is published right after
+      // the maxima, before this group's own codes, so it is normally there long before it is read.
       float sm_prev = -INFINITY;
       if (j > 0) {
-        ok = mbar_wait(bar(L::B_XCH + 4 * ((grp + kGroups - 1) % kGroups) + quad), ((j - 1) / kGroups) & 1,
-                       abort_flag, a.wait_budget);
-        if (!__all_sync(0xFFFFFFFFu, ok)) return false;
-        sm_prev = mx[row];
+        unsigned long long v = mx[row];
+        if (!__all_sync(0xFFFFFFFFu, (uint32_t)(v >> 32) == (uint32_t)(j - 1))) {
+          const long long t0 = clock64();
+          while (true) {
+            v = mx[row];
+            if (__all_sync(0xFFFFFFFFu, (uint32_t)(v >> 32) == (uint32_t)(j - 1))) break;
+            if (__any_sync(0xFFFFFFFFu, *abort_flag != 0 || clock64() - t0 > a.wait_budget)) return ok = false;
+          }
+        }
+        sm_prev = __uint_as_float((uint32_t)v);
       }
       const bool move = j == 0 || (mt_raw * c > sm_prev * c + tau);
       const float sm_new = move ? mt_raw : sm_prev;
-      if (j + 1 < TJ) {  // hand the max on as early as possible: the other group waits for it
-        mx[row] = sm_new;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_XCH + 4 * grp + quad));
-      }
+      if (j + 1 < TJ)  // hand the max on as early as possible: the other group waits for it
+        mx[row] = ((unsigned long long)(uint32_t)j << 32) | __float_as_uint(sm_new);
       codes(sm_new);
       const float m2 = sm_new * c;
       // O~ and l are rescaled by alpha = 2^(m_old - m_new) only when some row of the warp moves
