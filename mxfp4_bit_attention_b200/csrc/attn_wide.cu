@@ -475,6 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
         float* ds = reinterpret_cast<float*>(a.dump + dl.s) + ((size_t)j * 128 + row) * kBN;
         for (int i = 0; i < 128; i++) ds[i] = __uint_as_float(s[i]);
       }
+      // the hand-over slot is first read here, so that its latency overlaps the maxima (the value is
+      // normally there long before; the check below reads again until it is)
+      unsigned long long v0 = j > 0 ? mx[row] : 0ull;
       float gmax[4];
       group_maxima(s, gmax);
       const float mt_raw = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3]));
@@ -521,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       // the maxima, before this group's own codes, so it is normally there long before it is read.
       float sm_prev = -INFINITY;
       if (j > 0) {
-        unsigned long long v = mx[row];
+        unsigned long long v = v0;
         if (!__all_sync(0xFFFFFFFFu, (uint32_t)(v >> 32) == (uint32_t)(j - 1))) {
           const long long t0 = clock64();
           while (true) {
