@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       mbar_init(bar(L::B_KV_EMPTY + s), 1);
     }
     for (int i = 0; i < kSFullSlots; i++) mbar_init(bar(L::B_S_FULL + i), 1);
-    for (int b = 0; b < 2; b++) mbar_init(bar(L::B_S_FREE + b), 4);
+    for (int b = 0; b < 2; b++) mbar_init(bar(L::B_S_FREE + b), 128);  // every thread of a group
     for (int b = 0; b < kPBufs; b++) {
       mbar_init(bar(L::B_P_FULL + b), 4);
       mbar_init(bar(L::B_O_DONE + b), 1);
@@ -461,10 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1) mxattn_fwd_wide_kernel(const Attn
       const uint32_t sbuf = tl + L::T_S + 128 * (j & 1);
       uint32_t s[128];
       tmem_ld128_wait(sbuf, s);
-      // S(j) is in registers: the QK MMA of tile j+2 may overwrite the buffer
+      // S(j) is in registers: the QK MMA of tile j+2 may overwrite the buffer.  Each thread fences
+      // its own load and arrives (no warp barrier on the way to the maxima).
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_S_FREE + (j & 1)));
+      mbar_arrive(bar(L::B_S_FREE + (j & 1)));
       if (!FULL) {
         const int valid = kmax - j * kBN;  // this row's keys in the tile (may be <= 0)
 #pragma unroll
